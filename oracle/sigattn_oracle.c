@@ -1,0 +1,172 @@
+/*
+ * Plain fp64 CPU oracle for padding-aware bidirectional sigmoid attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link or
+ * call this file: only the test suite, the smoke check and the benchmark's CPU
+ * baseline use it.  It shares no code, header or constant with the CUDA path.
+ *
+ * What it computes (all arithmetic in double, on the exact input values):
+ *
+ *   gist.science summary, section 2.A (sigmoid attention mechanism):
+ *       O = sigma(Q K^T / sqrt(d) + b) V,  sigma(x) = 1 / (1 + e^-x),
+ *       applied element-wise with no row normalisation; alpha generalises
+ *       1/sqrt(d) as in the paper.rainbus.top summary, method step (2)
+ *       ("S = Q K^T alpha + b").
+ *   paper.rainbus.top summary, method steps (1)-(2): inputs are Z x L x H x D
+ *       with per-sample true lengths n_q, n_k; key positions at or beyond n_k
+ *       get -inf added, i.e. weight sigma = 0; query rows at or beyond n_q are
+ *       written as zero.
+ *   paper.rainbus.top summary, method step (4): dS = P (1 - P) (dO V^T);
+ *       dQ = alpha dS K; dK/dV by the transposed view: dK = alpha dS^T Q,
+ *       dV = P^T dO.  Padded query rows are constants (written as zero), so no
+ *       gradient flows from them: their dO is ignored.
+ *
+ * Readings where the pages are silent are listed in the design notes; here:
+ *   - the -inf mask is applied by selection (P = 0), never by adding -inf;
+ *   - sigma is the exact logistic function, not the tanh approximation the
+ *     kernel pages describe (the approximation is what the oracle judges).
+ *
+ * Layout of every tensor: [Z][L][H][D], contiguous; element (z,l,h,d) sits at
+ * ((z*L + l)*H + h)*D + d.  dtype 0 = bf16 (raw uint16 bits), 1 = fp32.
+ * Row lists are int64 triples (z, h, row).  Outputs are double, D per row.
+ *
+ * Parallelism: OpenMP over independent rows only; each row is summed in
+ * ascending index order, exactly as the definition reads.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* Exact widening of one stored element to double. */
+static double load_elem(const void *base, int dtype, int64_t idx) {
+    if (dtype == 0) {
+        uint16_t b = ((const uint16_t *)base)[idx];
+        uint32_t bits = ((uint32_t)b) << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)base)[idx];
+}
+
+static int64_t offset_of(int64_t z, int64_t l, int64_t h, int L, int H, int D) {
+    return ((z * L + l) * H + h) * (int64_t)D;
+}
+
+/* logistic function, gist.science summary section 2.A; both branches are the
+ * same closed form, written so that exp never overflows. */
+double oracle_sigmoid(double x) {
+    if (x >= 0.0) return 1.0 / (1.0 + exp(-x));
+    double e = exp(x);
+    return e / (1.0 + e);
+}
+
+/* its derivative as the pages state it: sigma'(x) = sigma(x) (1 - sigma(x)) */
+double oracle_sigmoid_grad(double x) {
+    double p = oracle_sigmoid(x);
+    return p * (1.0 - p);
+}
+
+/* score x_ij = alpha * sum_d Q[i,d] K[j,d] + b for one (z, h) */
+static double score(const void *q, const void *k, int dtype, int64_t z, int64_t h,
+                    int64_t i, int64_t j, int L, int H, int D, double alpha, double bias) {
+    int64_t qo = offset_of(z, i, h, L, H, D), ko = offset_of(z, j, h, L, H, D);
+    double s = 0.0;
+    for (int d = 0; d < D; ++d) s += load_elem(q, dtype, qo + d) * load_elem(k, dtype, ko + d);
+    return alpha * s + bias;
+}
+
+static double dot_rows(const void *a, const void *b, int dtype, int64_t z, int64_t h,
+                       int64_t i, int64_t j, int L, int H, int D) {
+    int64_t ao = offset_of(z, i, h, L, H, D), bo = offset_of(z, j, h, L, H, D);
+    double s = 0.0;
+    for (int d = 0; d < D; ++d) s += load_elem(a, dtype, ao + d) * load_elem(b, dtype, bo + d);
+    return s;
+}
+
+static int clamp_len(int n, int L) { return n < 0 ? 0 : (n > L ? L : n); }
+
+/* Forward rows: O[z, i, h, :] = [i < n_q] sum_{j < n_k} sigma(x_ij) V[z, j, h, :]. */
+void oracle_fwd_rows(const void *q, const void *k, const void *v, int dtype,
+                     int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
+                     double alpha, double bias, const int64_t *items, int64_t nitems,
+                     double *out) {
+    (void)Z;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t t = 0; t < nitems; ++t) {
+        int64_t z = items[3 * t], h = items[3 * t + 1], i = items[3 * t + 2];
+        double *o = out + t * D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        if (i >= n_q) continue;
+        for (int64_t j = 0; j < n_k; ++j) {
+            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
+            int64_t vo = offset_of(z, j, h, L, H, D);
+            for (int d = 0; d < D; ++d) o[d] += p * load_elem(v, dtype, vo + d);
+        }
+    }
+}
+
+/* dQ rows: dQ[z, i, h, :] = [i < n_q] alpha sum_{j < n_k} dS_ij K[z, j, h, :],
+ * dS_ij = P_ij (1 - P_ij) (dO_i . V_j). */
+void oracle_dq_rows(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                    int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
+                    double alpha, double bias, const int64_t *items, int64_t nitems,
+                    double *out) {
+    (void)Z;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t t = 0; t < nitems; ++t) {
+        int64_t z = items[3 * t], h = items[3 * t + 1], i = items[3 * t + 2];
+        double *g = out + t * D;
+        for (int d = 0; d < D; ++d) g[d] = 0.0;
+        int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        if (i >= n_q) continue;
+        for (int64_t j = 0; j < n_k; ++j) {
+            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
+            double dp = dot_rows(dout, v, dtype, z, h, i, j, L, H, D);
+            double ds = p * (1.0 - p) * dp;
+            int64_t ko = offset_of(z, j, h, L, H, D);
+            for (int d = 0; d < D; ++d) g[d] += ds * load_elem(k, dtype, ko + d);
+        }
+        for (int d = 0; d < D; ++d) g[d] *= alpha;
+    }
+}
+
+/* dK and dV rows for key j:
+ *   dV[z, j, h, :] = [j < n_k] sum_{i < n_q} P_ij dO[z, i, h, :]
+ *   dK[z, j, h, :] = [j < n_k] alpha sum_{i < n_q} dS_ij Q[z, i, h, :] */
+void oracle_dkdv_rows(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                      int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
+                      double alpha, double bias, const int64_t *items, int64_t nitems,
+                      double *dk_out, double *dv_out) {
+    (void)Z;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t t = 0; t < nitems; ++t) {
+        int64_t z = items[3 * t], h = items[3 * t + 1], j = items[3 * t + 2];
+        double *gk = dk_out + t * D, *gv = dv_out + t * D;
+        for (int d = 0; d < D; ++d) { gk[d] = 0.0; gv[d] = 0.0; }
+        int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        if (j >= n_k) continue;
+        for (int64_t i = 0; i < n_q; ++i) {
+            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
+            double dp = dot_rows(dout, v, dtype, z, h, i, j, L, H, D);
+            double ds = p * (1.0 - p) * dp;
+            int64_t qo = offset_of(z, i, h, L, H, D);
+            for (int d = 0; d < D; ++d) {
+                gv[d] += p * load_elem(dout, dtype, qo + d);
+                gk[d] += ds * load_elem(q, dtype, qo + d);
+            }
+        }
+        for (int d = 0; d < D; ++d) gk[d] *= alpha;
+    }
+}
+
+/* Number of OpenMP threads the oracle runs with (for reporting). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
