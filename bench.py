@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of padding-aware sigmoid attention (forward + backward) on B200.
+
+One step = one forward (sigattn_fwd) and one backward (sigattn_bwd: dQ kernel
++ dK/dV kernel) over one batch of the 16K / head-dim-128 kernel-benchmark
+workload without padding (Z=2, H=16, L=16384, D=128, bf16; paperlayer.ai
+summary, section 4).  The 25%-padding workload (Z=4, L=16384, n ~ U[8192,
+16384]) is measured the same way and reported beside it, with the padding
+loss.  Throughput counts valid-token FLOPs: 4 D H sum n_q n_k forward and 2.5x
+that backward (paperlayer.ai summary, appendix A.2).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs its own batch (weak scaling; the path shards
+over independent (z, h) problems with no collective); the time is the max over
+ranks.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd/bwd TFLOPS (valid tokens) at L=16K d=128, 0%/25% pad; % of B200 BF16 peak"
+HEADLINE = 3      # 16K, no padding
+PADDED = 4        # 16K, 25% padding
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(bf16=float(d["bf16_tflops"]), bf16_sustained=float(d["bf16_tflops_sustained"]),
+                    hbm=float(d["hbm_gbs"]), source="measured")
+    except Exception:
+        return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+
+def cpu_sample(w, rows: int, seed: int = 0):
+    """A bounded sample of one workload for the fp64 oracle: `rows` query rows
+    (forward + dQ) and `rows` key rows (dK, dV), spread over (z, h)."""
+    from padding_aware_sigmoid_b200 import workloads as W
+    inp = W.make_inputs(w) if w.Z * w.L * w.H * w.D <= 2 ** 27 else None
+    g = np.random.default_rng(seed)
+    n = W.lengths(w)
+    if inp is None:  # full-size tensors, drawn exactly as the GPU run draws them
+        inp = W.make_inputs(w)
+    z = g.integers(0, w.Z, size=rows)
+    h = g.integers(0, w.H, size=rows)
+    r = np.array([g.integers(0, max(int(n[zz]), 1)) for zz in z])
+    items = np.stack([z, h, r], axis=1).astype(np.int64)
+    # counted FLOPs of the sample: each row carries its n_k (resp. n_q) pairs
+    pairs = float(np.sum(n[z]))
+    counted = (1.0 + 2.5) * 4.0 * w.D * pairs
+    return inp, items, counted
+
+
+def run_oracle_step(inp, items):
+    import oracle
+    a = (inp["q"], inp["k"], inp["v"])
+    lens = (inp["seqlens_q"], inp["seqlens_k"], inp["alpha"], inp["bias"])
+    oracle.fwd_rows(*a, *lens, items)
+    oracle.dq_rows(*a, inp["dout"], *lens, items)
+    oracle.dkdv_rows(*a, inp["dout"], *lens, items)
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    from padding_aware_sigmoid_b200 import workloads as W
+    w = W.WORKLOADS[HEADLINE]
+    rows = 96
+    inp, items, counted = cpu_sample(w, rows)
+    for _ in range(max(args.warmup, 0)):
+        run_oracle_step(inp, items[:8])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run_oracle_step(inp, items)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = counted / dt / 1e12
+    cores = oracle.num_threads()
+    sample = (f"{rows} query rows (fwd + dQ) and {rows} key rows (dK, dV) per step, drawn from "
+              f"the {w.name} workload (Z={w.Z}, H={w.H}, L={w.L}, D={w.D})")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "Z": w.Z, "H": w.H, "L": w.L, "D": w.D,
+                   "lengths": "n_q = n_k = 16384", "parallelism": "single host process"},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+
+
+def make_device_inputs(w, device, seed_offset: int):
+    import torch
+    from padding_aware_sigmoid_b200 import workloads as W
+    n = W.lengths(w)
+    g = torch.Generator(device=device).manual_seed(1000 * w.index + seed_offset)
+    q, k, v, do = (torch.randn((w.Z, w.L, w.H, w.D), generator=g, device=device,
+                               dtype=torch.float32).mul_(w.qkv_scale if i < 3 else 1.0)
+                   .to(torch.bfloat16) for i in range(4))
+    nd = torch.as_tensor(n, dtype=torch.int32, device=device)
+    return dict(q=q, k=k, v=v, dout=do, nq=nd, nk=nd, n=n)
+
+
+def time_workload(sa, w, inp, steps, warmup, device, sampler=None):
+    """Times K steps (fwd + bwd) with CUDA events on the launching stream; also
+    the per-call durations of the forward, the dQ and the dK/dV kernels."""
+    import torch
+    st = torch.cuda.current_stream(device)
+    o = torch.empty_like(inp["q"])
+    dq, dk, dv = (torch.empty_like(inp["q"]) for _ in range(3))
+    args = (inp["q"], inp["k"], inp["v"])
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(st)
+        sa.fwd(*args, inp["nq"], inp["nk"], w.alpha, w.bias, out=o)
+        if ev is not None:
+            ev[1].record(st)
+        sa.bwd_dq(*args, inp["dout"], inp["nq"], inp["nk"], w.alpha, w.bias, dq=dq)
+        if ev is not None:
+            ev[2].record(st)
+        sa.bwd_dkdv(*args, inp["dout"], inp["nq"], inp["nk"], w.alpha, w.bias, dk=dk, dv=dv)
+        if ev is not None:
+            ev[3].record(st)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(st)
+    for i in range(steps):
+        step(evs[i])
+    end.record(st)
+    torch.cuda.synchronize(device)
+    total_ms = start.elapsed_time(end)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    dq_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    dkdv_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    assert sa.last_device_status(device) == 0
+    return total_ms / steps, fwd_ms, dq_ms, dkdv_ms
+
+
+def e2e_workload(sa, w, steps, warmup, device):
+    """Same step through the public API with host buffers: pinned host -> device
+    copies of Q, K, V, dO and the lengths, fwd + bwd, device -> host copies of O,
+    dQ, dK, dV, all inside the timed region."""
+    import torch
+    from padding_aware_sigmoid_b200 import workloads as W
+    hq, hk, hv, hdo = (torch.empty((w.Z, w.L, w.H, w.D), dtype=torch.bfloat16).pin_memory()
+                       for _ in range(4))
+    g = torch.Generator().manual_seed(7)
+    for t in (hq, hk, hv, hdo):
+        t.copy_(torch.randn(t.shape, generator=g).to(torch.bfloat16))
+    hn = torch.as_tensor(W.lengths(w), dtype=torch.int32).pin_memory()
+    outs = [torch.empty_like(hq).pin_memory() for _ in range(4)]
+    st = torch.cuda.current_stream(device)
+
+    def step():
+        q, k, v, do = (t.to(device, non_blocking=True) for t in (hq, hk, hv, hdo))
+        n = hn.to(device, non_blocking=True)
+        o = sa.fwd(q, k, v, n, n, w.alpha, w.bias)
+        dq, dk, dv = sa.bwd(q, k, v, do, n, n, w.alpha, w.bias)
+        for src, dst in zip((o, dq, dk, dv), outs):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(st)
+    for _ in range(steps):
+        step()
+    e.record(st)
+    torch.cuda.synchronize(device)
+    ms = s.elapsed_time(e) / steps
+    h2d = 4 * hq.numel() * 2 + hn.numel() * 4
+    d2h = 4 * hq.numel() * 2
+    return ms, h2d, d2h
+
+
+def our_arm(args, world, rank, local):
+    import torch
+    import padding_aware_sigmoid_b200 as sa
+    from padding_aware_sigmoid_b200 import workloads as W
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    pk = peaks()
+    w3, w4 = W.WORKLOADS[HEADLINE], W.WORKLOADS[PADDED]
+    f3 = W.fwd_flops_valid(W.lengths(w3), W.lengths(w3), w3.H, w3.D)
+    f4 = W.fwd_flops_valid(W.lengths(w4), W.lengths(w4), w4.H, w4.D)
+    f4_pad = W.fwd_flops_padded(w4.Z, w4.L, w4.H, w4.D)
+
+    inp3 = make_device_inputs(w3, device, rank)
+    barrier(world)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize(device)
+        step_ms, fwd_ms, dq_ms, dkdv_ms = time_workload(sa, w3, inp3, args.steps, args.warmup,
+                                                        device)
+    step_ms = max_over_ranks(step_ms, world, device)
+    barrier(world)
+    del inp3
+    inp4 = make_device_inputs(w4, device, rank)
+    step4_ms, fwd4_ms, dq4_ms, dkdv4_ms = time_workload(sa, w4, inp4, max(args.steps // 2, 3),
+                                                         args.warmup, device)
+    step4_ms = max_over_ranks(step4_ms, world, device)
+    del inp4
+    torch.cuda.empty_cache()
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_workload(sa, w3, max(args.steps // 4, 3), 2, device)
+        e2e_ms = max_over_ranks(e2e_ms, world, device)
+        e2e = {"value": world * f3 * 3.5 / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        rows = 1024
+        inp_cpu, items, counted = cpu_sample(w3, rows, seed=1)
+        t0 = time.perf_counter()
+        run_oracle_step(inp_cpu, items)
+        dt = time.perf_counter() - t0
+        cpu = {"value": counted / dt / 1e12, "unit": "TFLOPS", "cores": oracle.num_threads(),
+               "kind": "oracle", "seconds": dt,
+               "sample": f"{rows} query rows (fwd + dQ) and {rows} key rows (dK, dV) of the "
+                         f"{w3.name} workload, fp64, counted with the same FLOP convention"}
+
+    if rank != 0:
+        return
+    fwd_tf = f3 / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = 2.5 * f3 / ((dq_ms + dkdv_ms) * 1e-3) / 1e12
+    step_tf = world * 3.5 * f3 / (step_ms * 1e-3) / 1e12
+    fwd4_tf = f4 / (fwd4_ms * 1e-3) / 1e12
+    bwd4_tf = 2.5 * f4 / ((dq4_ms + dkdv4_ms) * 1e-3) / 1e12
+    # dominant kernel: the longest of the three per step
+    kernels = {"fwd": (fwd_ms, f3), "bwd_dkdv": (dkdv_ms, 8.0 / 4.0 * f3),
+               "bwd_dq": (dq_ms, 6.0 / 4.0 * f3)}
+    dom = max(kernels, key=lambda k: kernels[k][0])
+    dom_ms, dom_flops = kernels[dom]
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    traffic = _ncu_traffic(dom)
+    line = {
+        "metric": METRIC,
+        "value": step_tf,
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w3.name, "Z": w3.Z, "H": w3.H, "L": w3.L, "D": w3.D,
+            "lengths": "n_q = n_k = 16384", "global_batch": world * w3.Z, "seq_len": w3.L,
+            "parallelism": f"dp{world} over independent (z, h) problems, no collective",
+            "l2": "inputs larger than L2: each of Q, K, V, dO is %.0f MB" % (
+                w3.Z * w3.L * w3.H * w3.D * 2 / 1e6),
+            "sigmoid_mode": "tanh" if sa.get_sigmoid_mode() == sa.SIGMOID_TANH else "exp",
+        },
+        "fwd_tflops": fwd_tf,
+        "bwd_tflops": bwd_tf,
+        "fwd_ms": fwd_ms, "bwd_dq_ms": dq_ms, "bwd_dkdv_ms": dkdv_ms,
+        "fwd_pct_of_peak": 100.0 * fwd_tf / pk["bf16"],
+        "bwd_pct_of_peak": 100.0 * bwd_tf / pk["bf16"],
+        "pad25": {
+            "workload": w4.name, "lengths": [int(x) for x in W.lengths(w4)],
+            "fwd_tflops": fwd4_tf, "bwd_tflops": bwd4_tf,
+            "fwd_tflops_padded_flops": f4_pad / (fwd4_ms * 1e-3) / 1e12,
+            "fwd_padding_loss_pct": 100.0 * (1.0 - fwd4_tf / fwd_tf),
+            "bwd_padding_loss_pct": 100.0 * (1.0 - bwd4_tf / bwd_tf),
+            "ms_per_step": step4_ms,
+        },
+        "roofline": {
+            "kernel": dom, "bound": "tensor", "achieved": achieved, "peak": pk["bf16"],
+            "unit": "TFLOP/s", "frac": achieved / pk["bf16"], "traffic": traffic,
+            "peak_kind": f"{pk['source']} bf16 burst (cuBLAS 8192^3)",
+            "frac_of_sustained": achieved / pk["bf16_sustained"],
+            "flops_per_launch": dom_flops,
+        },
+        "clocks": clk.summary(),
+        "gpu_launches": 3 * args.steps,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary of the same kernel, if
+    one exists for the current build; None otherwise."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(kernel)
+    except Exception:
+        return None
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            reference_arm(args, world, rank)
+        else:
+            our_arm(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,162 @@
+/*
+ * sigattn — padding-aware bidirectional sigmoid self-attention on NVIDIA B200
+ * (sm_100a).  C ABI of libsigattn.so.
+ *
+ * The operation (gist.science summary of "Better Models, Faster Training:
+ * Sigmoid Attention for single-cell Foundation Models", section 2.A, and the
+ * paper.rainbus.top summary of the same paper, method steps (1)-(5)):
+ *
+ *   S  = alpha * Q K^T + b                        per sample z and head h
+ *   P  = sigma(S) with P[i, j] = 0 for keys j >= n_k(z)   (the "-inf" mask)
+ *   O  = P V, and O[i, :] = 0 for query rows i >= n_q(z)
+ *   dS = P (1 - P) (dO V^T)          (padded query rows carry no gradient)
+ *   dQ = alpha dS K,  dK = alpha dS^T Q,  dV = P^T dO
+ *
+ * sigma is the logistic function 1 / (1 + e^-x); there is no row
+ * normalisation.  The backward recomputes P (method step (5)); it needs
+ * neither O nor any saved statistic.
+ *
+ * Layout of every tensor argument: [Z][L][H][D], contiguous, row-major:
+ * element (z, l, h, d) at ((z * L + l) * H + h) * D + d.  Z = batch, L =
+ * padded length, H = heads, D = head dimension.  Base pointers must be
+ * 16-byte aligned (every pointer PyTorch allocates is).
+ *
+ * Sequence lengths are int32[Z] arrays in DEVICE memory (n_q and n_k may
+ * differ).  They are read by the kernels, not by the host.  Values outside
+ * [0, L] are clamped on the device and flag SIGATTN_ERR_SEQLEN_RANGE in the
+ * device status word (see sigattn_last_device_status).
+ *
+ * Ownership: the caller owns and allocates every buffer; calls allocate
+ * nothing per call.  The library lazily allocates, once per device, a small
+ * device status buffer that lives until process exit.
+ *
+ * Asynchrony: every compute call enqueues its kernels on `stream` (a
+ * cudaStream_t passed as void*; NULL = the legacy default stream) and
+ * returns without synchronising.  The return code covers argument
+ * validation and launch errors only; errors detected on the device (bounded
+ * waits that ran out, clamped lengths) accumulate in the device status word.
+ *
+ * Precision: SIGATTN_BF16 inputs/outputs run on the tcgen05 tensor cores
+ * with fp32 accumulation in tensor memory (P and dS are rounded to bf16
+ * before their second matmul).  SIGATTN_FP32 runs an fp32 CUDA-core path
+ * meant for accuracy checks, not speed.
+ */
+#ifndef SIGATTN_H
+#define SIGATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SIGATTN_OK = 0,
+    SIGATTN_ERR_INVALID_ARG = 1,          /* null pointer, non-positive size, ... */
+    SIGATTN_ERR_UNSUPPORTED_HEADDIM = 2,  /* D not in {64, 128} */
+    SIGATTN_ERR_UNSUPPORTED_DTYPE = 3,
+    SIGATTN_ERR_UNSUPPORTED_DEVICE = 4,   /* bf16 path needs compute capability 10.0 */
+    SIGATTN_ERR_MISALIGNED = 5,           /* a base pointer is not 16-byte aligned */
+    SIGATTN_ERR_CUDA = 6,                 /* a CUDA runtime/driver call failed */
+    SIGATTN_ERR_TIMEOUT = 7,              /* device: a bounded wait ran out */
+    SIGATTN_ERR_SEQLEN_RANGE = 8          /* device: a length was outside [0, L] */
+} sigattn_status;
+
+typedef enum {
+    SIGATTN_BF16 = 0,
+    SIGATTN_FP32 = 1
+} sigattn_dtype;
+
+/* How the bf16 kernels evaluate sigma in registers.
+ * SIGATTN_SIGMOID_TANH: sigma(x) = 0.5 tanh(x / 2) + 0.5 with the hardware
+ *   tanh.approx.f32 (paper.rainbus.top summary, method step (3)); one MUFU
+ *   operation per score.
+ * SIGATTN_SIGMOID_EXP: u = e^-|x| with one hardware ex2.approx, then
+ *   g = 1/(1+u) by a degree-4 minimax polynomial on the FMA pipe (relative
+ *   error < 3.4e-4) and sigma = g (x >= 0) or u g (x < 0); one MUFU
+ *   operation per score and relative accuracy in both tails.
+ * The fp32 path always uses the exact library expf. */
+typedef enum {
+    SIGATTN_SIGMOID_TANH = 0,
+    SIGATTN_SIGMOID_EXP = 1
+} sigattn_sigmoid_mode;
+
+/* Forward: O = [i < n_q] * sum_{j < n_k} sigma(alpha q_i . k_j + b) v_j.
+ * q, k, v: [Z][L][H][D] inputs (device, read only).  o: [Z][L][H][D] output
+ * (device); every element is written, padded query rows as exact zeros.
+ * D in {64, 128}; any L >= 1 (partial tiles are masked); Z, H >= 1.
+ * Errors: SIGATTN_ERR_INVALID_ARG, _UNSUPPORTED_HEADDIM, _UNSUPPORTED_DTYPE,
+ * _UNSUPPORTED_DEVICE, _MISALIGNED, _CUDA.  On error nothing is launched. */
+sigattn_status sigattn_fwd(const void *q, const void *k, const void *v, void *o,
+                           const int32_t *seqlens_q, const int32_t *seqlens_k,
+                           int Z, int L, int H, int D, float alpha, float bias,
+                           sigattn_dtype dtype, void *stream);
+
+/* Backward: given dout = dL/dO, writes dq, dk, dv (each [Z][L][H][D],
+ * device, fully written; rows at or beyond n_q (dq) or n_k (dk, dv) are exact
+ * zeros).  dout rows at or beyond n_q are ignored.  Launches a dQ kernel and
+ * a dK/dV kernel on `stream`; neither uses atomics.  Same errors as
+ * sigattn_fwd. */
+sigattn_status sigattn_bwd(const void *q, const void *k, const void *v, const void *dout,
+                           void *dq, void *dk, void *dv,
+                           const int32_t *seqlens_q, const int32_t *seqlens_k,
+                           int Z, int L, int H, int D, float alpha, float bias,
+                           sigattn_dtype dtype, void *stream);
+
+/* The two halves of sigattn_bwd, for callers that want to run them on
+ * separate streams (they only read q, k, v, dout and write disjoint
+ * outputs) or time them apart.  sigattn_bwd_dq writes dq; sigattn_bwd_dkdv
+ * writes dk and dv.  Arguments, layout and errors as sigattn_bwd. */
+sigattn_status sigattn_bwd_dq(const void *q, const void *k, const void *v, const void *dout,
+                              void *dq, const int32_t *seqlens_q, const int32_t *seqlens_k,
+                              int Z, int L, int H, int D, float alpha, float bias,
+                              sigattn_dtype dtype, void *stream);
+sigattn_status sigattn_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
+                                void *dk, void *dv, const int32_t *seqlens_q,
+                                const int32_t *seqlens_k, int Z, int L, int H, int D,
+                                float alpha, float bias, sigattn_dtype dtype, void *stream);
+
+/* Selects how later bf16 calls in this process evaluate sigma (process-wide,
+ * default SIGATTN_SIGMOID_EXP; see sigattn_sigmoid_mode).  Returns
+ * SIGATTN_ERR_INVALID_ARG for an unknown mode. */
+sigattn_status sigattn_set_sigmoid_mode(sigattn_sigmoid_mode mode);
+sigattn_sigmoid_mode sigattn_get_sigmoid_mode(void);
+
+/* Evaluates the kernels' own device sigma routine for `mode` on n fp32
+ * values: y[i] = sigma(x[i]) and, if dy != NULL, dy[i] = sigma'(x[i]) as
+ * the backward kernels form it.  x, y, dy are device arrays of n floats.
+ * Used to measure the error of the in-register sigma against fp64. */
+sigattn_status sigattn_sigmoid_eval(const float *x, float *y, float *dy, int64_t n,
+                                    sigattn_sigmoid_mode mode, void *stream);
+
+/* Reads and clears the current device's status word: synchronises `stream`
+ * and returns SIGATTN_OK or the first device-side error recorded since the
+ * last call (SIGATTN_ERR_TIMEOUT or SIGATTN_ERR_SEQLEN_RANGE). */
+sigattn_status sigattn_last_device_status(void *stream);
+
+/* Bound, in nanoseconds, on every wait inside the bf16 kernels (default
+ * 4e9).  A wait that runs out records SIGATTN_ERR_TIMEOUT, the kernel
+ * abandons its work, frees its tensor memory and exits. */
+sigattn_status sigattn_set_wait_timeout_ns(uint64_t ns);
+
+/* Launches a one-CTA kernel whose only job is to wait on a barrier that
+ * nothing signals, bounded by timeout_ns; it must return with
+ * SIGATTN_ERR_TIMEOUT recorded in the status word and leave the context
+ * usable.  Exercises the failure path of the bounded waits. */
+sigattn_status sigattn_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
+
+/* Text of the CUDA error behind the most recent SIGATTN_ERR_CUDA returned
+ * by any call in this process (static string; "no error" if none). */
+const char *sigattn_last_cuda_error(void);
+
+/* Human-readable name of a status code (static string). */
+const char *sigattn_status_string(sigattn_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int sigattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIGATTN_H */

@@ -1,0 +1,257 @@
+"""Padding-aware bidirectional sigmoid self-attention for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over ``libsigattn.so`` (C ABI in ``include/sigattn.h``).
+PyTorch supplies device memory and the current CUDA stream; every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback:
+calling any op without the built library or without a CUDA device raises.
+
+    O = sigma(alpha Q K^T + b) V   (keys >= n_k masked, query rows >= n_q zero)
+
+Tensors are [Z, L, H, D] (batch, padded length, heads, head dim), contiguous,
+bf16 (tensor-core path) or fp32 (accuracy path); ``seqlens_q`` / ``seqlens_k``
+are int32 [Z] on the same device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "SigattnError", "fwd", "bwd", "sigmoid_eval", "set_sigmoid_mode", "get_sigmoid_mode",
+    "last_device_status", "set_wait_timeout_ns", "selftest_wait_timeout", "status_string",
+    "version", "library_path", "load_library", "SIGMOID_TANH", "SIGMOID_EXP", "EXPORTS",
+    "SigmoidAttention", "bwd_dq", "bwd_dkdv", "last_cuda_error",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsigattn.so")
+_lock = threading.Lock()
+_lib = None
+
+SIGMOID_TANH = 0
+SIGMOID_EXP = 1
+_BF16, _FP32 = 0, 1
+
+STATUS_NAMES = {
+    0: "SIGATTN_OK", 1: "SIGATTN_ERR_INVALID_ARG", 2: "SIGATTN_ERR_UNSUPPORTED_HEADDIM",
+    3: "SIGATTN_ERR_UNSUPPORTED_DTYPE", 4: "SIGATTN_ERR_UNSUPPORTED_DEVICE",
+    5: "SIGATTN_ERR_MISALIGNED", 6: "SIGATTN_ERR_CUDA", 7: "SIGATTN_ERR_TIMEOUT",
+    8: "SIGATTN_ERR_SEQLEN_RANGE",
+}
+
+# every symbol include/sigattn.h declares
+EXPORTS = (
+    "sigattn_fwd", "sigattn_bwd", "sigattn_bwd_dq", "sigattn_bwd_dkdv",
+    "sigattn_set_sigmoid_mode", "sigattn_get_sigmoid_mode", "sigattn_sigmoid_eval",
+    "sigattn_last_device_status", "sigattn_set_wait_timeout_ns", "sigattn_selftest_wait_timeout",
+    "sigattn_last_cuda_error", "sigattn_status_string", "sigattn_version",
+)
+
+
+class SigattnError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: str = ""):
+        self.code = int(code)
+        msg = f"{where}: {STATUS_NAMES.get(self.code, self.code)}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Loads libsigattn.so (built in-tree by ``padding_aware_sigmoid_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"libsigattn.so is not built ({_LIB_PATH}); run "
+                              "`python -m padding_aware_sigmoid_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, ci, cf, i64, u64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64,
+                                ctypes.c_uint64)
+        lib.sigattn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf, ci, vp]
+        lib.sigattn_fwd.restype = ci
+        lib.sigattn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf,
+                                    ci, vp]
+        lib.sigattn_bwd.restype = ci
+        lib.sigattn_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf, ci, vp]
+        lib.sigattn_bwd_dq.restype = ci
+        lib.sigattn_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf,
+                                         ci, vp]
+        lib.sigattn_bwd_dkdv.restype = ci
+        lib.sigattn_last_cuda_error.restype = ctypes.c_char_p
+        lib.sigattn_set_sigmoid_mode.argtypes = [ci]
+        lib.sigattn_set_sigmoid_mode.restype = ci
+        lib.sigattn_get_sigmoid_mode.restype = ci
+        lib.sigattn_sigmoid_eval.argtypes = [vp, vp, vp, i64, ci, vp]
+        lib.sigattn_sigmoid_eval.restype = ci
+        lib.sigattn_last_device_status.argtypes = [vp]
+        lib.sigattn_last_device_status.restype = ci
+        lib.sigattn_set_wait_timeout_ns.argtypes = [u64]
+        lib.sigattn_set_wait_timeout_ns.restype = ci
+        lib.sigattn_selftest_wait_timeout.argtypes = [u64, vp]
+        lib.sigattn_selftest_wait_timeout.restype = ci
+        lib.sigattn_status_string.argtypes = [ci]
+        lib.sigattn_status_string.restype = ctypes.c_char_p
+        lib.sigattn_version.restype = ci
+        _lib = lib
+        return lib
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        detail = last_cuda_error() if code == 6 else ""
+        raise SigattnError(code, where, detail)
+
+
+def _stream_ptr(t) -> int:
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return _BF16
+    if t.dtype == torch.float32:
+        return _FP32
+    raise TypeError(f"sigattn takes bf16 or fp32 tensors, got {t.dtype}")
+
+
+def _check_inputs(tensors, seqlens):
+    import torch
+    ref = tensors[0]
+    if ref.dim() != 4:
+        raise ValueError("tensors must be [Z, L, H, D]")
+    for t in tensors:
+        if not t.is_cuda:
+            raise ValueError("sigattn tensors must live on a CUDA device (no CPU fallback)")
+        if t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+            raise ValueError("all tensors must share shape, dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [Z, L, H, D]")
+    for s in seqlens:
+        if not (s.is_cuda and s.dtype == torch.int32 and s.dim() == 1 and s.shape[0] == ref.shape[0]
+                and s.is_contiguous() and s.device == ref.device):
+            raise ValueError("seqlens must be contiguous int32 [Z] tensors on the tensors' device")
+
+
+def fwd(q, k, v, seqlens_q, seqlens_k, alpha: float, bias: float, out=None):
+    """O = [i < n_q] sum_{j < n_k} sigma(alpha q_i . k_j + bias) v_j, [Z, L, H, D]."""
+    import torch
+    _check_inputs([q, k, v], [seqlens_q, seqlens_k])
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_inputs([q, out], [])
+    Z, L, H, D = (int(s) for s in q.shape)
+    lib = load_library()
+    _check(lib.sigattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                           seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, L, H, D, float(alpha),
+                           float(bias), _dtype_code(q), _stream_ptr(q)), "sigattn_fwd")
+    return out
+
+
+def bwd(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, dq=None, dk=None,
+        dv=None):
+    """(dQ, dK, dV) given dout = dLoss/dO; P is recomputed, O is not needed."""
+    import torch
+    _check_inputs([q, k, v, dout], [seqlens_q, seqlens_k])
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_inputs([q, dq, dk, dv], [])
+    Z, L, H, D = (int(s) for s in q.shape)
+    lib = load_library()
+    _check(lib.sigattn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), seqlens_q.data_ptr(),
+                           seqlens_k.data_ptr(), Z, L, H, D, float(alpha), float(bias),
+                           _dtype_code(q), _stream_ptr(q)), "sigattn_bwd")
+    return dq, dk, dv
+
+
+def bwd_dq(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, dq=None):
+    """dQ only (the dQ kernel of the backward)."""
+    import torch
+    _check_inputs([q, k, v, dout], [seqlens_q, seqlens_k])
+    dq = torch.empty_like(q) if dq is None else dq
+    _check_inputs([q, dq], [])
+    Z, L, H, D = (int(s) for s in q.shape)
+    _check(load_library().sigattn_bwd_dq(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+        seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, L, H, D, float(alpha), float(bias),
+        _dtype_code(q), _stream_ptr(q)), "sigattn_bwd_dq")
+    return dq
+
+
+def bwd_dkdv(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, dk=None, dv=None):
+    """(dK, dV) only (the dK/dV kernel of the backward)."""
+    import torch
+    _check_inputs([q, k, v, dout], [seqlens_q, seqlens_k])
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_inputs([q, dk, dv], [])
+    Z, L, H, D = (int(s) for s in q.shape)
+    _check(load_library().sigattn_bwd_dkdv(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+        seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, L, H, D, float(alpha), float(bias),
+        _dtype_code(q), _stream_ptr(q)), "sigattn_bwd_dkdv")
+    return dk, dv
+
+
+def last_cuda_error() -> str:
+    return load_library().sigattn_last_cuda_error().decode()
+
+
+def sigmoid_eval(x, mode: int):
+    """(sigma(x), sigma'(x)) as evaluated in the bf16 kernels' registers (fp32 CUDA x)."""
+    import torch
+    if not (x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()):
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    dy = torch.empty_like(x)
+    _check(load_library().sigattn_sigmoid_eval(x.data_ptr(), y.data_ptr(), dy.data_ptr(),
+                                               x.numel(), int(mode), _stream_ptr(x)),
+           "sigattn_sigmoid_eval")
+    return y, dy
+
+
+def set_sigmoid_mode(mode: int):
+    _check(load_library().sigattn_set_sigmoid_mode(int(mode)), "sigattn_set_sigmoid_mode")
+
+
+def get_sigmoid_mode() -> int:
+    return int(load_library().sigattn_get_sigmoid_mode())
+
+
+def last_device_status(device=None) -> int:
+    """Reads and clears the device status word (synchronises the current stream)."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return int(load_library().sigattn_last_device_status(
+            torch.cuda.current_stream(dev).cuda_stream))
+
+
+def set_wait_timeout_ns(ns: int):
+    _check(load_library().sigattn_set_wait_timeout_ns(int(ns)), "sigattn_set_wait_timeout_ns")
+
+
+def selftest_wait_timeout(ns: int):
+    import torch
+    _check(load_library().sigattn_selftest_wait_timeout(
+        int(ns), torch.cuda.current_stream().cuda_stream), "sigattn_selftest_wait_timeout")
+
+
+def status_string(code: int) -> str:
+    return load_library().sigattn_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return int(load_library().sigattn_version())
+
+
+from .autograd import SigmoidAttention  # noqa: E402  (needs the functions above)

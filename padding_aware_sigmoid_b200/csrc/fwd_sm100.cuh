@@ -1,0 +1,315 @@
+// Forward kernel: O = sigma(alpha Q K^T + b) V with key padding masked and
+// padded query rows zeroed (gist.science summary, section 2.A;
+// paper.rainbus.top summary, method steps (1)-(3)).
+//
+// One CTA owns two 128-row query tiles of one (z, h) and streams the key/value
+// tiles j < ceil(n_k / 128) through shared memory; key tiles wholly in padding
+// are never loaded, query tiles wholly in padding are written as zeros
+// without any load (the pages' block-sparse skip, paperlayer.ai summary,
+// section 4).
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q tiles once, then K_j / V_j into a ring of stages
+//   warp 1      owns TMEM; one thread issues every tcgen05.mma
+//   warps 4-7   sigma warpgroup of query tile 0 (thread = query row)
+//   warps 8-11  sigma warpgroup of query tile 1
+// Tensor memory (512 columns, fp32):
+//   [0,128) S0   [128,256) S1   [256,256+D) O0   [256+D,256+2D) O1
+// P_t (bf16, two per column) overwrites the first 64 columns of S_t and is the
+// TMEM-resident A operand of O_t += P_t V_j, so P never touches shared memory.
+//
+// Per key tile j the MMA thread issues S0 = Q0 K_j^T, S1 = Q1 K_j^T, then
+// O0 += P0 V_j, O1 += P1 V_j as the warpgroups publish P.  S_t of tile j+1 is
+// issued only after O_t += P_t V_j has completed (P_t aliases S_t); the other
+// query tile's work fills the tensor pipe meanwhile.
+#pragma once
+
+#include "sm100.cuh"
+#include "sigmoid.cuh"
+
+namespace sigattn {
+
+struct FwdParams {
+    __nv_bfloat16 *o;
+    const int *seqlens_q;
+    const int *seqlens_k;
+    int L, H;
+    float alpha, bias;
+    int *status;
+    uint64_t timeout_ns;
+};
+
+template <int D, int STAGES>
+struct FwdLayout {
+    static constexpr int BM = 128;                 // query rows per tile
+    static constexpr int BN = 128;                 // keys per tile
+    static constexpr int NSUB = D / 64;            // 64-column swizzle atoms per row
+    static constexpr int SUB_BYTES = 128 * 64 * 2; // one [128][64] bf16 atom column
+    static constexpr int TILE_BYTES = NSUB * SUB_BYTES;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
+    // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
+    // pv_done[2], drain
+    static constexpr int NBAR = 1 + 4 * STAGES + 7;
+    static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM + 8;
+    static constexpr int BYTES = OFF_ABORT + 8;
+    static constexpr int SMEM_ALLOC = BYTES + 1024;  // slack to align the base to 1 KiB
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+    static_assert(COL_O1 + D <= TMEM_COLS, "TMEM budget");
+};
+
+__device__ __forceinline__ uint8_t *align_1k(uint8_t *p) {
+    uint32_t a = smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// Waits that never consult the abort flag: used to drain in-flight async work
+// before the CTA releases its shared and tensor memory.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return;
+    uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) return;
+    }
+}
+
+template <int D, int MODE, int STAGES>
+__global__ void __launch_bounds__(384, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+    using Lay = FwdLayout<D, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align_1k(smem_raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::OFF_BAR);
+    uint64_t *q_full = bars;
+    uint64_t *k_full = bars + 1;
+    uint64_t *k_empty = k_full + STAGES;
+    uint64_t *v_full = k_empty + STAGES;
+    uint64_t *v_empty = v_full + STAGES;
+    uint64_t *s_full = v_empty + STAGES;
+    uint64_t *p_full = s_full + 2;
+    uint64_t *pv_done = p_full + 2;
+    uint64_t *drain = pv_done + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
+
+    const int warp = warp_id(), lane = lane_id();
+    const int z = blockIdx.z, h = blockIdx.y;
+    const int qtile0 = blockIdx.x * 2;
+    const int L = p.L;
+
+    int nq = p.seqlens_q[z], nk = p.seqlens_k[z];
+    if (nq < 0 || nq > L || nk < 0 || nk > L) {
+        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
+        nq = min(max(nq, 0), L);
+        nk = min(max(nk, 0), L);
+    }
+    const int ntiles = (qtile0 * Lay::BM < nq ? 1 : 0) + ((qtile0 + 1) * Lay::BM < nq ? 1 : 0);
+    const int nkv = (nk + Lay::BN - 1) / Lay::BN;
+    const bool work = ntiles > 0 && nkv > 0;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], 128);
+            mbar_init(&pv_done[t], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Lay::TMEM_COLS);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (work && lane == 0) {
+            uint8_t *sQ = smem + Lay::OFF_Q;
+            uint8_t *sK = smem + Lay::OFF_K;
+            uint8_t *sV = smem + Lay::OFF_V;
+            mbar_arrive_expect_tx(q_full, ntiles * Lay::TILE_BYTES);
+            for (int t = 0; t < ntiles; ++t)
+                for (int s = 0; s < Lay::NSUB; ++s)
+                    tma_load_4d(&tmQ, q_full, sQ + t * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
+                                64 * s, h, (qtile0 + t) * Lay::BM, z);
+            int issued_k = 0, issued_v = 0;
+            for (int j = 0; j < nkv; ++j) {
+                const int st = j % STAGES, round = j / STAGES;
+                if (j >= STAGES && !mbar_wait(&k_empty[st], (round - 1) & 1, wctx)) break;
+                mbar_arrive_expect_tx(&k_full[st], Lay::TILE_BYTES);
+                for (int s = 0; s < Lay::NSUB; ++s)
+                    tma_load_4d(&tmK, &k_full[st], sK + st * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
+                                64 * s, h, j * Lay::BN, z);
+                issued_k = j + 1;
+                if (j >= STAGES && !mbar_wait(&v_empty[st], (round - 1) & 1, wctx)) break;
+                mbar_arrive_expect_tx(&v_full[st], Lay::TILE_BYTES);
+                for (int s = 0; s < Lay::NSUB; ++s)
+                    tma_load_4d(&tmV, &v_full[st], sV + st * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
+                                64 * s, h, j * Lay::BN, z);
+                issued_v = j + 1;
+            }
+            // Every issued load must land before the CTA's shared memory is released.
+            mbar_wait_drain(q_full, 0, p.timeout_ns);
+            for (int j = (issued_k > STAGES ? issued_k - STAGES : 0); j < issued_k; ++j)
+                mbar_wait_drain(&k_full[j % STAGES], (j / STAGES) & 1, p.timeout_ns);
+            for (int j = (issued_v > STAGES ? issued_v - STAGES : 0); j < issued_v; ++j)
+                mbar_wait_drain(&v_full[j % STAGES], (j / STAGES) & 1, p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (work && lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(128, Lay::BN, false, false);
+            const uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+            const uint32_t sQ = smem_u32(smem + Lay::OFF_Q);
+            const uint32_t sK = smem_u32(smem + Lay::OFF_K);
+            const uint32_t sV = smem_u32(smem + Lay::OFF_V);
+            bool ok = mbar_wait(q_full, 0, wctx);
+            for (int j = 0; ok && j < nkv; ++j) {
+                const int st = j % STAGES, round = j / STAGES;
+                if (!(ok = mbar_wait(&k_full[st], round & 1, wctx))) break;
+                const uint32_t kbase = sK + st * Lay::TILE_BYTES;
+                for (int t = 0; t < ntiles; ++t) {
+                    if (j > 0 && !(ok = mbar_wait(&pv_done[t], (j - 1) & 1, wctx))) break;
+                    tc_fence_after();
+                    const uint32_t qbase = sQ + t * Lay::TILE_BYTES;
+                    const uint32_t d_tmem = tmem + (t ? Lay::COL_S1 : Lay::COL_S0);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
+                        mma_ss(d_tmem, smem_desc_sw128(qbase + koff, 16, 1024),
+                               smem_desc_sw128(kbase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&s_full[t]);
+                }
+                if (!ok) break;
+                mma_commit(&k_empty[st]);
+                if (!(ok = mbar_wait(&v_full[st], round & 1, wctx))) break;
+                const uint32_t vbase = sV + st * Lay::TILE_BYTES;
+                for (int t = 0; t < ntiles; ++t) {
+                    if (!(ok = mbar_wait(&p_full[t], j & 1, wctx))) break;
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem + (t ? Lay::COL_O1 : Lay::COL_O0);
+                    const uint32_t a_tmem = tmem + (t ? Lay::COL_S1 : Lay::COL_S0);
+#pragma unroll
+                    for (int kk = 0; kk < Lay::BN / 16; ++kk) {
+                        // 16 keys per step: 8 packed TMEM columns of P, 16 rows of V
+                        mma_ts(d_tmem, a_tmem + kk * 8,
+                               smem_desc_sw128(vbase + kk * 16 * 128, Lay::SUB_BYTES, 1024),
+                               idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&pv_done[t]);
+                }
+                if (!ok) break;
+                mma_commit(&v_empty[st]);
+            }
+            // No MMA may still be running when TMEM is released.
+            mma_commit(drain);
+            mbar_wait_drain(drain, 0, p.timeout_ns);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ sigma warpgroups
+        const int t = (warp - 4) >> 2;
+        const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+        const int row = (qtile0 + t) * Lay::BM + quarter * 32 + lane;
+        const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_bits + (t ? Lay::COL_S1 : Lay::COL_S0);
+        const uint32_t tO = tmem + lane_bits + (t ? Lay::COL_O1 : Lay::COL_O0);
+        const size_t row_stride = static_cast<size_t>(p.H) * D;
+        __nv_bfloat16 *orow = p.o + (static_cast<size_t>(z) * L + row) * row_stride +
+                              static_cast<size_t>(h) * D;
+        const bool active = work && t < ntiles;
+        bool ok = true;
+        if (active) {
+            const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
+            for (int j = 0; j < nkv; ++j) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wctx));
+                if (!ok) break;
+                tc_fence_after();
+                const int kbase = j * Lay::BN;
+                const bool partial = kbase + Lay::BN > nk;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + 32 * c, r);
+                                        uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 pr = sigma2<MODE>(
+                            scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
+                        float p0 = pr.x, p1 = pr.y;
+                        if (partial) {
+                            const int key = kbase + 32 * c + 2 * i;
+                            if (key >= nk) p0 = 0.0f;
+                            if (key + 1 >= nk) p1 = 0.0f;
+                        }
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    // P columns [16c, 16c+16) lie inside S columns already read.
+                    tmem_st16(tS + 16 * c, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&p_full[t]);
+            }
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[t], (nkv - 1) & 1, wctx));
+            if (ok) {
+                tc_fence_after();
+                const bool valid = row < nq;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tO + 32 * c, r);
+                                        if (row < L) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            uint4 w;
+                            w.x = valid ? pack_bf16x2(__uint_as_float(r[8 * v4 + 0]), __uint_as_float(r[8 * v4 + 1])) : 0u;
+                            w.y = valid ? pack_bf16x2(__uint_as_float(r[8 * v4 + 2]), __uint_as_float(r[8 * v4 + 3])) : 0u;
+                            w.z = valid ? pack_bf16x2(__uint_as_float(r[8 * v4 + 4]), __uint_as_float(r[8 * v4 + 5])) : 0u;
+                            w.w = valid ? pack_bf16x2(__uint_as_float(r[8 * v4 + 6]), __uint_as_float(r[8 * v4 + 7])) : 0u;
+                            dst[v4] = w;
+                        }
+                    }
+                }
+            }
+        } else if (row < L) {
+            // query tile wholly in padding, or no valid key: exact zeros, no loads
+            uint4 *dst = reinterpret_cast<uint4 *>(orow);
+#pragma unroll
+            for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, Lay::TMEM_COLS);
+    }
+}
+
+}  // namespace sigattn

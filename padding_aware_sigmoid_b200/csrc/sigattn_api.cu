@@ -1,0 +1,353 @@
+// C ABI of libsigattn.so (declared in include/sigattn.h): argument checks,
+// TMA tensor-map encoding and kernel launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/sigattn.h"
+#include "bwd_sm100.cuh"
+#include "fp32_simt.cuh"
+#include "fwd_sm100.cuh"
+
+namespace {
+
+using namespace sigattn;
+
+constexpr int kMaxDevices = 64;
+constexpr int kFwdStagesD128 = 2;
+constexpr int kFwdStagesD64 = 4;
+constexpr int kBwdStages = 2;
+
+std::mutex g_mu;
+int *g_status[kMaxDevices] = {};          // device status word per device (lazy, never freed)
+int g_cc_major[kMaxDevices] = {};         // 0 = not queried yet
+std::atomic<int> g_sigmoid_mode{kSigmoidExp};
+std::atomic<uint64_t> g_timeout_ns{4000000000ull};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<int> g_last_cuda_error{0};
+
+// Records the failing call's error (and clears the runtime's last error).
+sigattn_status cuda_fail(cudaError_t e = cudaSuccess) {
+    cudaError_t last = cudaGetLastError();
+    g_last_cuda_error.store(static_cast<int>(e != cudaSuccess ? e : last));
+    return SIGATTN_ERR_CUDA;
+}
+
+// Current device, its compute capability and its status word.
+sigattn_status device_state(int *dev, int *cc_major, int **status) {
+    if (cudaGetDevice(dev) != cudaSuccess) return cuda_fail();
+    if (*dev < 0 || *dev >= kMaxDevices) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_cc_major[*dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess)
+            return cuda_fail();
+        g_cc_major[*dev] = major * 10 + minor;
+    }
+    if (g_status[*dev] == nullptr) {
+        int *s = nullptr;
+        if (cudaMalloc(&s, 64) != cudaSuccess) return cuda_fail();
+        if (cudaMemset(s, 0, 64) != cudaSuccess) return cuda_fail();
+        g_status[*dev] = s;
+    }
+    *cc_major = g_cc_major[*dev];
+    *status = g_status[*dev];
+    return SIGATTN_OK;
+}
+
+sigattn_status get_encoder() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode != nullptr) return SIGATTN_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return cuda_fail();
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return SIGATTN_OK;
+}
+
+// [Z][L][H][D] bf16 viewed as a 4-D tensor (D, H, L, Z), boxes of 64 x 1 x 128 x 1
+// elements with 128-byte swizzle: one box is one [128 rows][64 cols] operand atom.
+sigattn_status encode_bf16_map(CUtensorMap *m, const void *base, int Z, int L, int H, int D) {
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(Z)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                             static_cast<cuuint64_t>(L) * H * D * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error.store(10000 + static_cast<int>(r));
+        return SIGATTN_ERR_CUDA;
+    }
+    return SIGATTN_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sigattn_status check_shape(int Z, int L, int H, int D, sigattn_dtype dtype, bool *empty) {
+    if (Z < 0 || L < 0 || H < 0) return SIGATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SIGATTN_ERR_UNSUPPORTED_HEADDIM;
+    if (dtype != SIGATTN_BF16 && dtype != SIGATTN_FP32) return SIGATTN_ERR_UNSUPPORTED_DTYPE;
+    if (H > 65535 || Z > 65535) return SIGATTN_ERR_INVALID_ARG;
+    *empty = (Z == 0 || L == 0 || H == 0);
+    return SIGATTN_OK;
+}
+
+template <typename... KArgs, typename... Args>
+sigattn_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t stream, Args... args) {
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return SIGATTN_OK;
+}
+
+template <int D, int MODE>
+sigattn_status fwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                        const FwdParams &p, int Z, int L, int H, cudaStream_t st) {
+    constexpr int S = D == 128 ? kFwdStagesD128 : kFwdStagesD64;
+    dim3 grid((L + 255) / 256, H, Z);
+    return launch(fwd_kernel<D, MODE, S>, grid, dim3(384), FwdLayout<D, S>::SMEM_ALLOC, st, mq, mk,
+                  mv, p);
+}
+
+enum BwdParts : int { kPartDq = 1, kPartDkdv = 2 };
+
+template <int D, int MODE>
+sigattn_status bwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                        const CUtensorMap &mdo, const BwdParams &p, int Z, int L, int H,
+                        int parts, cudaStream_t st) {
+    dim3 grid((L + 127) / 128, H, Z);
+    constexpr size_t smem = BwdLayout<D, kBwdStages>::SMEM_ALLOC;
+    if (parts & kPartDq) {
+        sigattn_status s = launch(bwd_dq_kernel<D, MODE, kBwdStages>, grid, dim3(384), smem, st, mq,
+                                  mk, mv, mdo, p);
+        if (s != SIGATTN_OK) return s;
+    }
+    if (parts & kPartDkdv)
+        return launch(bwd_dkdv_kernel<D, MODE, kBwdStages>, grid, dim3(384), smem, st, mq, mk, mv,
+                      mdo, p);
+    return SIGATTN_OK;
+}
+
+// Shared body of sigattn_bwd, sigattn_bwd_dq and sigattn_bwd_dkdv.
+sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void *dout, void *dq,
+                        void *dk, void *dv, const int32_t *seqlens_q, const int32_t *seqlens_k,
+                        int Z, int L, int H, int D, float alpha, float bias, sigattn_dtype dtype,
+                        void *stream, int parts) {
+    bool empty = false;
+    sigattn_status s = check_shape(Z, L, H, D, dtype, &empty);
+    if (s != SIGATTN_OK) return s;
+    if (empty) return SIGATTN_OK;
+    if (!q || !k || !v || !dout || !seqlens_q || !seqlens_k) return SIGATTN_ERR_INVALID_ARG;
+    if (((parts & kPartDq) && !dq) || ((parts & kPartDkdv) && (!dk || !dv)))
+        return SIGATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
+        ((parts & kPartDq) && !aligned16(dq)) ||
+        ((parts & kPartDkdv) && (!aligned16(dk) || !aligned16(dv))))
+        return SIGATTN_ERR_MISALIGNED;
+    int dev, cc;
+    int *status;
+    if ((s = device_state(&dev, &cc, &status)) != SIGATTN_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == SIGATTN_FP32) {
+        F32Params p{static_cast<const float *>(q),    static_cast<const float *>(k),
+                    static_cast<const float *>(v),    static_cast<const float *>(dout),
+                    nullptr,                          static_cast<float *>(dq),
+                    static_cast<float *>(dk),         static_cast<float *>(dv),
+                    seqlens_q,                        seqlens_k,
+                    Z, L, H, alpha, bias, status};
+        const int64_t rows = static_cast<int64_t>(Z) * L * H;
+        dim3 grid(static_cast<unsigned>((rows + 7) / 8));
+        if (parts & kPartDq) {
+            s = D == 64 ? launch(f32_dq_kernel<64>, grid, dim3(256), 0, st, p)
+                        : launch(f32_dq_kernel<128>, grid, dim3(256), 0, st, p);
+            if (s != SIGATTN_OK) return s;
+        }
+        if (parts & kPartDkdv)
+            return D == 64 ? launch(f32_dkdv_kernel<64>, grid, dim3(256), 0, st, p)
+                           : launch(f32_dkdv_kernel<128>, grid, dim3(256), 0, st, p);
+        return SIGATTN_OK;
+    }
+    if (cc != 100) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
+    if ((s = get_encoder()) != SIGATTN_OK) return s;
+    CUtensorMap mq, mk, mv, mdo;
+    if ((s = encode_bf16_map(&mq, q, Z, L, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mdo, dout, Z, L, H, D)) != SIGATTN_OK) return s;
+    BwdParams p{static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
+                static_cast<__nv_bfloat16 *>(dv), seqlens_q, seqlens_k, L, H, alpha, bias, status,
+                g_timeout_ns.load()};
+    const int mode = g_sigmoid_mode.load();
+    if (D == 128)
+        return mode == kSigmoidTanh
+                   ? bwd_bf16<128, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, L, H, parts, st)
+                   : bwd_bf16<128, kSigmoidExp>(mq, mk, mv, mdo, p, Z, L, H, parts, st);
+    return mode == kSigmoidTanh ? bwd_bf16<64, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, L, H, parts, st)
+                                : bwd_bf16<64, kSigmoidExp>(mq, mk, mv, mdo, p, Z, L, H, parts, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+sigattn_status sigattn_fwd(const void *q, const void *k, const void *v, void *o,
+                           const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int L, int H,
+                           int D, float alpha, float bias, sigattn_dtype dtype, void *stream) {
+    bool empty = false;
+    sigattn_status s = check_shape(Z, L, H, D, dtype, &empty);
+    if (s != SIGATTN_OK) return s;
+    if (empty) return SIGATTN_OK;
+    if (!q || !k || !v || !o || !seqlens_q || !seqlens_k) return SIGATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return SIGATTN_ERR_MISALIGNED;
+    int dev, cc;
+    int *status;
+    if ((s = device_state(&dev, &cc, &status)) != SIGATTN_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == SIGATTN_FP32) {
+        F32Params p{static_cast<const float *>(q), static_cast<const float *>(k),
+                    static_cast<const float *>(v), nullptr, static_cast<float *>(o), nullptr,
+                    nullptr, nullptr, seqlens_q, seqlens_k, Z, L, H, alpha, bias, status};
+        const int64_t rows = static_cast<int64_t>(Z) * L * H;
+        dim3 grid(static_cast<unsigned>((rows + 7) / 8));
+        return D == 64 ? launch(f32_fwd_kernel<64>, grid, dim3(256), 0, st, p)
+                       : launch(f32_fwd_kernel<128>, grid, dim3(256), 0, st, p);
+    }
+    if (cc != 100) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
+    if ((s = get_encoder()) != SIGATTN_OK) return s;
+    CUtensorMap mq, mk, mv;
+    if ((s = encode_bf16_map(&mq, q, Z, L, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
+    FwdParams p{static_cast<__nv_bfloat16 *>(o), seqlens_q, seqlens_k, L, H, alpha, bias, status,
+                g_timeout_ns.load()};
+    const int mode = g_sigmoid_mode.load();
+    if (D == 128)
+        return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
+                                    : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
+    return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
+                                : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
+}
+
+sigattn_status sigattn_bwd(const void *q, const void *k, const void *v, const void *dout, void *dq,
+                           void *dk, void *dv, const int32_t *seqlens_q, const int32_t *seqlens_k,
+                           int Z, int L, int H, int D, float alpha, float bias,
+                           sigattn_dtype dtype, void *stream) {
+    return bwd_impl(q, k, v, dout, dq, dk, dv, seqlens_q, seqlens_k, Z, L, H, D, alpha, bias, dtype,
+                    stream, kPartDq | kPartDkdv);
+}
+
+sigattn_status sigattn_bwd_dq(const void *q, const void *k, const void *v, const void *dout,
+                              void *dq, const int32_t *seqlens_q, const int32_t *seqlens_k, int Z,
+                              int L, int H, int D, float alpha, float bias, sigattn_dtype dtype,
+                              void *stream) {
+    return bwd_impl(q, k, v, dout, dq, nullptr, nullptr, seqlens_q, seqlens_k, Z, L, H, D, alpha,
+                    bias, dtype, stream, kPartDq);
+}
+
+sigattn_status sigattn_bwd_dkdv(const void *q, const void *k, const void *v, const void *dout,
+                                void *dk, void *dv, const int32_t *seqlens_q,
+                                const int32_t *seqlens_k, int Z, int L, int H, int D, float alpha,
+                                float bias, sigattn_dtype dtype, void *stream) {
+    return bwd_impl(q, k, v, dout, nullptr, dk, dv, seqlens_q, seqlens_k, Z, L, H, D, alpha, bias,
+                    dtype, stream, kPartDkdv);
+}
+
+sigattn_status sigattn_set_sigmoid_mode(sigattn_sigmoid_mode mode) {
+    if (mode != SIGATTN_SIGMOID_TANH && mode != SIGATTN_SIGMOID_EXP) return SIGATTN_ERR_INVALID_ARG;
+    g_sigmoid_mode.store(mode == SIGATTN_SIGMOID_TANH ? kSigmoidTanh : kSigmoidExp);
+    return SIGATTN_OK;
+}
+
+sigattn_sigmoid_mode sigattn_get_sigmoid_mode(void) {
+    return g_sigmoid_mode.load() == kSigmoidTanh ? SIGATTN_SIGMOID_TANH : SIGATTN_SIGMOID_EXP;
+}
+
+sigattn_status sigattn_sigmoid_eval(const float *x, float *y, float *dy, int64_t n,
+                                    sigattn_sigmoid_mode mode, void *stream) {
+    if (n < 0 || (n > 0 && (!x || !y))) return SIGATTN_ERR_INVALID_ARG;
+    if (mode != SIGATTN_SIGMOID_TANH && mode != SIGATTN_SIGMOID_EXP) return SIGATTN_ERR_INVALID_ARG;
+    if (n == 0) return SIGATTN_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dim3 grid(static_cast<unsigned>((n + 255) / 256));
+    return mode == SIGATTN_SIGMOID_TANH
+               ? launch(sigmoid_eval_kernel<kSigmoidTanh>, grid, dim3(256), 0, st, x, y, dy, n)
+               : launch(sigmoid_eval_kernel<kSigmoidExp>, grid, dim3(256), 0, st, x, y, dy, n);
+}
+
+sigattn_status sigattn_last_device_status(void *stream) {
+    int dev, cc;
+    int *status;
+    sigattn_status s = device_state(&dev, &cc, &status);
+    if (s != SIGATTN_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int host = 0;
+    if (cudaMemcpyAsync(&host, status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return cuda_fail();
+    if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_fail();
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return cuda_fail();
+    if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_fail();
+    return static_cast<sigattn_status>(host);
+}
+
+sigattn_status sigattn_set_wait_timeout_ns(uint64_t ns) {
+    if (ns == 0) return SIGATTN_ERR_INVALID_ARG;
+    g_timeout_ns.store(ns);
+    return SIGATTN_OK;
+}
+
+sigattn_status sigattn_selftest_wait_timeout(uint64_t timeout_ns, void *stream) {
+    if (timeout_ns == 0 || timeout_ns > 10000000000ull) return SIGATTN_ERR_INVALID_ARG;
+    int dev, cc;
+    int *status;
+    sigattn_status s = device_state(&dev, &cc, &status);
+    if (s != SIGATTN_OK) return s;
+    return launch(wait_timeout_selftest_kernel, dim3(1), dim3(32), 0,
+                  static_cast<cudaStream_t>(stream), status, timeout_ns);
+}
+
+const char *sigattn_status_string(sigattn_status s) {
+    switch (s) {
+        case SIGATTN_OK: return "SIGATTN_OK";
+        case SIGATTN_ERR_INVALID_ARG: return "SIGATTN_ERR_INVALID_ARG";
+        case SIGATTN_ERR_UNSUPPORTED_HEADDIM: return "SIGATTN_ERR_UNSUPPORTED_HEADDIM";
+        case SIGATTN_ERR_UNSUPPORTED_DTYPE: return "SIGATTN_ERR_UNSUPPORTED_DTYPE";
+        case SIGATTN_ERR_UNSUPPORTED_DEVICE: return "SIGATTN_ERR_UNSUPPORTED_DEVICE";
+        case SIGATTN_ERR_MISALIGNED: return "SIGATTN_ERR_MISALIGNED";
+        case SIGATTN_ERR_CUDA: return "SIGATTN_ERR_CUDA";
+        case SIGATTN_ERR_TIMEOUT: return "SIGATTN_ERR_TIMEOUT";
+        case SIGATTN_ERR_SEQLEN_RANGE: return "SIGATTN_ERR_SEQLEN_RANGE";
+    }
+    return "SIGATTN_UNKNOWN_STATUS";
+}
+
+const char *sigattn_last_cuda_error(void) {
+    const int e = g_last_cuda_error.load();
+    if (e == 0) return "no error";
+    if (e >= 10000) return "cuTensorMapEncodeTiled failed";
+    return cudaGetErrorString(static_cast<cudaError_t>(e));
+}
+
+int sigattn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,99 @@
+"""CPU checks of the C ABI: the library builds, loads, and exports exactly the
+entry points include/sigattn.h declares; host-side argument validation works
+without a GPU; the product path has no CPU fallback and never touches the
+oracle."""
+import ctypes
+import os
+import re
+import shutil
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sigattn.h")
+PKG = os.path.join(ROOT, "padding_aware_sigmoid_b200")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sigattn_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from padding_aware_sigmoid_b200 import build
+    if not os.path.exists(build.OUT):
+        if shutil.which("nvcc") is None and not os.path.exists("/usr/local/cuda/bin/nvcc"):
+            pytest.skip("nvcc unavailable and library not built")
+        build.build()
+    import padding_aware_sigmoid_b200 as sa
+    return sa.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    assert "sigattn_fwd" in names and "sigattn_bwd" in names
+    import padding_aware_sigmoid_b200 as sa
+    assert sorted(sa.EXPORTS) == names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), f"{name} not exported by libsigattn.so"
+
+
+def test_status_strings_and_version(lib):
+    import padding_aware_sigmoid_b200 as sa
+    for code, name in sa.STATUS_NAMES.items():
+        assert sa.status_string(code) == name
+    assert sa.version() >= 100
+
+
+def test_host_validation_needs_no_gpu(lib):
+    vp = ctypes.c_void_p
+    dummy = vp(16)
+    # unsupported head dim is rejected before any device call
+    assert lib.sigattn_fwd(dummy, dummy, dummy, dummy, dummy, dummy, 1, 128, 1, 96, 1.0, 0.0, 0,
+                           None) == 2
+    # negative sizes and null pointers
+    assert lib.sigattn_fwd(dummy, dummy, dummy, dummy, dummy, dummy, -1, 128, 1, 64, 1.0, 0.0, 0,
+                           None) == 1
+    assert lib.sigattn_fwd(None, dummy, dummy, dummy, dummy, dummy, 1, 128, 1, 64, 1.0, 0.0, 0,
+                           None) == 1
+    assert lib.sigattn_bwd(dummy, dummy, dummy, dummy, dummy, dummy, None, dummy, dummy, 1, 128, 1,
+                           64, 1.0, 0.0, 0, None) == 1
+    # unknown dtype
+    assert lib.sigattn_fwd(dummy, dummy, dummy, dummy, dummy, dummy, 1, 128, 1, 64, 1.0, 0.0, 7,
+                           None) == 3
+    # misaligned base pointer
+    odd = vp(16 + 2)
+    assert lib.sigattn_fwd(odd, dummy, dummy, dummy, dummy, dummy, 1, 128, 1, 64, 1.0, 0.0, 0,
+                           None) == 5
+    # empty problems are a no-op
+    assert lib.sigattn_fwd(dummy, dummy, dummy, dummy, dummy, dummy, 0, 128, 1, 64, 1.0, 0.0, 0,
+                           None) == 0
+    # sigmoid mode switch
+    assert lib.sigattn_set_sigmoid_mode(5) == 1
+    old = lib.sigattn_get_sigmoid_mode()
+    assert lib.sigattn_set_sigmoid_mode(0) == 0 and lib.sigattn_get_sigmoid_mode() == 0
+    assert lib.sigattn_set_sigmoid_mode(old) == 0
+    assert lib.sigattn_set_wait_timeout_ns(0) == 1
+
+
+def test_no_cpu_fallback(lib):
+    import torch
+    import padding_aware_sigmoid_b200 as sa
+    x = torch.zeros((1, 128, 1, 64), dtype=torch.bfloat16)
+    n = torch.full((1,), 128, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        sa.fwd(x, x, x, n, n, 1.0, 0.0)
+
+
+def test_product_path_never_imports_the_oracle():
+    for dirpath, _, files in os.walk(PKG):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "sigattn_oracle" not in text, f
