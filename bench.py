@@ -45,6 +45,10 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=["fwd", "dq", "dkdv", "all"], default=None,
+                    help="launch only this kernel (profiling runs; prints timings, no JSON line)")
+    ap.add_argument("--shape", default="2,16,4096,128", help="Z,H,L,D for --only")
+    ap.add_argument("--sigmoid-mode", choices=["exp", "tanh"], default=None)
     return ap.parse_args()
 
 
@@ -156,11 +160,9 @@ def cpu_sample(w, rows: int, seed: int = 0):
     """A bounded sample of one workload for the fp64 oracle: `rows` query rows
     (forward + dQ) and `rows` key rows (dK, dV), spread over (z, h)."""
     from padding_aware_sigmoid_b200 import workloads as W
-    inp = W.make_inputs(w) if w.Z * w.L * w.H * w.D <= 2 ** 27 else None
+    inp = W.make_inputs(w)
     g = np.random.default_rng(seed)
     n = W.lengths(w)
-    if inp is None:  # full-size tensors, drawn exactly as the GPU run draws them
-        inp = W.make_inputs(w)
     z = g.integers(0, w.Z, size=rows)
     h = g.integers(0, w.H, size=rows)
     r = np.array([g.integers(0, max(int(n[zz]), 1)) for zz in z])
@@ -429,8 +431,51 @@ def _ncu_traffic(kernel: str):
         return None
 
 
+def only_kernel(args):
+    """Profiling helper: W warm-up and K timed launches of one kernel on a
+    Z,H,L,D problem with full lengths, bf16, alpha = 1/sqrt(D), b = -ln L."""
+    import torch
+    import padding_aware_sigmoid_b200 as sa
+    Z, H, L, D = (int(x) for x in args.shape.split(","))
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    q, k, v, do = (torch.randn((Z, L, H, D), generator=g, device=dev).to(torch.bfloat16)
+                   for _ in range(4))
+    n = torch.full((Z,), L, dtype=torch.int32, device=dev)
+    alpha, bias = 1.0 / math.sqrt(D), -math.log(L)
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    calls = {
+        "fwd": lambda: sa.fwd(q, k, v, n, n, alpha, bias, out=o),
+        "dq": lambda: sa.bwd_dq(q, k, v, do, n, n, alpha, bias, dq=dq),
+        "dkdv": lambda: sa.bwd_dkdv(q, k, v, do, n, n, alpha, bias, dk=dk, dv=dv),
+    }
+    names = list(calls) if args.only == "all" else [args.only]
+    flops = 4.0 * D * H * Z * L * L
+    per = {"fwd": flops, "dq": 1.5 * flops, "dkdv": 2.0 * flops}
+    for name in names:
+        for _ in range(args.warmup):
+            calls[name]()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            calls[name]()
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / args.steps
+        print(json.dumps({"kernel": name, "shape": [Z, H, L, D], "ms": ms,
+                          "tflops_executed": per[name] / ms / 1e9}), flush=True)
+    assert sa.last_device_status() == 0
+
+
 def main():
     args = parse()
+    if args.sigmoid_mode is not None:
+        import padding_aware_sigmoid_b200 as sa
+        sa.set_sigmoid_mode(sa.SIGMOID_TANH if args.sigmoid_mode == "tanh" else sa.SIGMOID_EXP)
+    if args.only is not None:
+        only_kernel(args)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -117,7 +117,7 @@ sigattn_status sigattn_bwd_dkdv(const void *q, const void *k, const void *v, con
                                 float alpha, float bias, sigattn_dtype dtype, void *stream);
 
 /* Selects how later bf16 calls in this process evaluate sigma (process-wide,
- * default SIGATTN_SIGMOID_EXP; see sigattn_sigmoid_mode).  Returns
+ * default SIGATTN_SIGMOID_TANH, the pages' form; see sigattn_sigmoid_mode).  Returns
  * SIGATTN_ERR_INVALID_ARG for an unknown mode. */
 sigattn_status sigattn_set_sigmoid_mode(sigattn_sigmoid_mode mode);
 sigattn_sigmoid_mode sigattn_get_sigmoid_mode(void);

@@ -51,8 +51,8 @@ struct FwdLayout {
     static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
     // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-    // pv_done[2], drain
-    static constexpr int NBAR = 1 + 4 * STAGES + 7;
+    // pv_done[2], drain, turn[2]
+    static constexpr int NBAR = 1 + 4 * STAGES + 9;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
     static constexpr int BYTES = OFF_ABORT + 8;
@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t *p_full = s_full + 2;
     uint64_t *pv_done = p_full + 2;
     uint64_t *drain = pv_done + 2;
+    uint64_t *turn = drain + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -126,6 +127,8 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&pv_done[t], 1);
         }
         mbar_init(drain, 1);
+        mbar_init(&turn[0], 128);
+        mbar_init(&turn[1], 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -186,44 +189,59 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t sQ = smem_u32(smem + Lay::OFF_Q);
             const uint32_t sK = smem_u32(smem + Lay::OFF_K);
             const uint32_t sV = smem_u32(smem + Lay::OFF_V);
-            bool ok = mbar_wait(q_full, 0, wctx);
-            for (int j = 0; ok && j < nkv; ++j) {
-                const int st = j % STAGES, round = j / STAGES;
-                if (!(ok = mbar_wait(&k_full[st], round & 1, wctx))) break;
-                const uint32_t kbase = sK + st * Lay::TILE_BYTES;
-                for (int t = 0; t < ntiles; ++t) {
-                    if (j > 0 && !(ok = mbar_wait(&pv_done[t], (j - 1) & 1, wctx))) break;
-                    tc_fence_after();
-                    const uint32_t qbase = sQ + t * Lay::TILE_BYTES;
-                    const uint32_t d_tmem = tmem + (t ? Lay::COL_S1 : Lay::COL_S0);
+            // S_t = Q_t K_j^T into TMEM columns of tile t
+            auto issue_s = [&](int t, uint32_t kbase) {
+                const uint32_t qbase = sQ + t * Lay::TILE_BYTES;
+                const uint32_t d_tmem = tmem + (t ? Lay::COL_S1 : Lay::COL_S0);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                        mma_ss(d_tmem, smem_desc_sw128(qbase + koff, 16, 1024),
-                               smem_desc_sw128(kbase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&s_full[t]);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
+                    mma_ss(d_tmem, smem_desc_sw128(qbase + koff, 16, 1024),
+                           smem_desc_sw128(kbase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
                 }
-                if (!ok) break;
-                mma_commit(&k_empty[st]);
-                if (!(ok = mbar_wait(&v_full[st], round & 1, wctx))) break;
-                const uint32_t vbase = sV + st * Lay::TILE_BYTES;
+                mma_commit(&s_full[t]);
+            };
+            // O_t += P_t V_j, P_t read from TMEM (16 keys = 8 packed columns per step)
+            auto issue_pv = [&](int t, uint32_t vbase, bool first) {
+                const uint32_t d_tmem = tmem + (t ? Lay::COL_O1 : Lay::COL_O0);
+                const uint32_t a_tmem = tmem + (t ? Lay::COL_S1 : Lay::COL_S0);
+#pragma unroll
+                for (int kk = 0; kk < Lay::BN / 16; ++kk)
+                    mma_ts(d_tmem, a_tmem + kk * 8,
+                           smem_desc_sw128(vbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_o,
+                           (!first || kk > 0) ? 1u : 0u);
+                mma_commit(&pv_done[t]);
+            };
+            // Order per key tile j: PV0_j, S0_{j+1}, PV1_j, S1_{j+1}.  Tile 0's next
+            // scores never wait for tile 1's P, so the two sigma warpgroups can
+            // alternate while the tensor pipe works on the other tile.  S_t of
+            // j+1 overwrites P_t of j, so it is issued only after PV_t_j completed.
+            bool ok = mbar_wait(q_full, 0, wctx) && mbar_wait(&k_full[0], 0, wctx);
+            if (ok) {
+                tc_fence_after();
+                for (int t = 0; t < ntiles; ++t) issue_s(t, sK);
+                mma_commit(&k_empty[0]);
+            }
+            for (int j = 0; ok && j < nkv; ++j) {
+                const int stv = j % STAGES;
+                const int stk = (j + 1) % STAGES;
+                const bool more = j + 1 < nkv;
+                const uint32_t vbase = sV + stv * Lay::TILE_BYTES;
+                const uint32_t knext = sK + stk * Lay::TILE_BYTES;
+                if (!(ok = mbar_wait(&v_full[stv], (j / STAGES) & 1, wctx))) break;
                 for (int t = 0; t < ntiles; ++t) {
                     if (!(ok = mbar_wait(&p_full[t], j & 1, wctx))) break;
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem + (t ? Lay::COL_O1 : Lay::COL_O0);
-                    const uint32_t a_tmem = tmem + (t ? Lay::COL_S1 : Lay::COL_S0);
-#pragma unroll
-                    for (int kk = 0; kk < Lay::BN / 16; ++kk) {
-                        // 16 keys per step: 8 packed TMEM columns of P, 16 rows of V
-                        mma_ts(d_tmem, a_tmem + kk * 8,
-                               smem_desc_sw128(vbase + kk * 16 * 128, Lay::SUB_BYTES, 1024),
-                               idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    issue_pv(t, vbase, j == 0);
+                    if (t == ntiles - 1) mma_commit(&v_empty[stv]);
+                    if (more) {
+                        if (t == 0 && !(ok = mbar_wait(&k_full[stk], ((j + 1) / STAGES) & 1, wctx))) break;
+                        if (!(ok = mbar_wait(&pv_done[t], j & 1, wctx))) break;
+                        tc_fence_after();
+                        issue_s(t, knext);
+                        if (t == ntiles - 1) mma_commit(&k_empty[stk]);
                     }
-                    mma_commit(&pv_done[t]);
                 }
-                if (!ok) break;
-                mma_commit(&v_empty[st]);
             }
             // No MMA may still be running when TMEM is released.
             mma_commit(drain);
@@ -244,35 +262,51 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         if (active) {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
+            const bool pingpong = ntiles == 2;
             for (int j = 0; j < nkv; ++j) {
+                // The two warpgroups take turns (tile 0 first) so that each sigma
+                // phase has the MUFU to itself while the tensor pipe runs the other
+                // tile's P.V and next scores.
+                if (pingpong && (t == 1 || j > 0)) {
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&turn[t], (t == 0 ? j - 1 : j) & 1, wctx));
+                    if (!ok) break;
+                }
                 ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wctx));
                 if (!ok) break;
                 tc_fence_after();
-                const int kbase = j * Lay::BN;
-                const bool partial = kbase + Lay::BN > nk;
+                const int kvalid = nk - j * Lay::BN;   // keys of this tile below n_k
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + 32 * c, r);
-                                        uint32_t pk[16];
+                for (int half = 0; half < 2; ++half) {
+                    // 64 scores of this row per TMEM read: two exposed load
+                    // latencies per tile
+                    uint32_t r[64];
+                    tmem_ld64(tS + 64 * half, r);
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
+                    for (int i = 0; i < 32; ++i) {
+                        const int c = 64 * half + 2 * i;
                         const float2 pr = sigma2<MODE>(
                             scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
-                        float p0 = pr.x, p1 = pr.y;
-                        if (partial) {
-                            const int key = kbase + 32 * c + 2 * i;
-                            if (key >= nk) p0 = 0.0f;
-                            if (key + 1 >= nk) p1 = 0.0f;
-                        }
-                        pk[i] = pack_bf16x2(p0, p1);
+                        pk[i] = pack_bf16x2_rh(pr.x, pr.y);
                     }
-                    // P columns [16c, 16c+16) lie inside S columns already read.
-                    tmem_st16(tS + 16 * c, pk);
+                    if (kvalid < Lay::BN) {
+                        // last tile: keys at or beyond n_k weigh exactly zero
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int c = 64 * half + 2 * i;
+                            const uint32_t lo = c < kvalid ? 0x0000FFFFu : 0u;
+                            const uint32_t hi = c + 1 < kvalid ? 0xFFFF0000u : 0u;
+                            pk[i] &= (lo | hi);
+                        }
+                    }
+                    // P columns [32 half, 32 half + 32) lie over S columns already read
+                    tmem_st32(tS + 32 * half, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[t]);
+                if (pingpong) mbar_arrive(&turn[t ^ 1]);
             }
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[t], (nkv - 1) & 1, wctx));
             if (ok) {

@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstdio>
 #include <mutex>
 
 #include "../../include/sigattn.h"
@@ -24,7 +25,7 @@ constexpr int kBwdStages = 2;
 std::mutex g_mu;
 int *g_status[kMaxDevices] = {};          // device status word per device (lazy, never freed)
 int g_cc_major[kMaxDevices] = {};         // 0 = not queried yet
-std::atomic<int> g_sigmoid_mode{kSigmoidExp};
+std::atomic<int> g_sigmoid_mode{kSigmoidTanh};
 std::atomic<uint64_t> g_timeout_ns{4000000000ull};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_last_cuda_error{0};
@@ -38,8 +39,14 @@ sigattn_status cuda_fail(cudaError_t e = cudaSuccess) {
 
 // Current device, its compute capability and its status word.
 sigattn_status device_state(int *dev, int *cc_major, int **status) {
-    if (cudaGetDevice(dev) != cudaSuccess) return cuda_fail();
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e);
     if (*dev < 0 || *dev >= kMaxDevices) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
+    // Makes the device's primary context current in the calling thread: the
+    // tensor-map encoder is a driver call and needs one (a fresh thread, such
+    // as PyTorch's autograd worker, may not have one yet).
+    e = cudaSetDevice(*dev);
+    if (e != cudaSuccess) return cuda_fail(e);
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_cc_major[*dev] == 0) {
         int major = 0, minor = 0;
@@ -344,7 +351,11 @@ const char *sigattn_status_string(sigattn_status s) {
 const char *sigattn_last_cuda_error(void) {
     const int e = g_last_cuda_error.load();
     if (e == 0) return "no error";
-    if (e >= 10000) return "cuTensorMapEncodeTiled failed";
+    if (e >= 10000) {
+        static thread_local char buf[64];
+        snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (CUresult %d)", e - 10000);
+        return buf;
+    }
     return cudaGetErrorString(static_cast<cudaError_t>(e));
 }
 

@@ -51,14 +51,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// One poll of the barrier; a thread whose phase has not completed may be
+// suspended by the hardware for up to `kSuspendHintNs` (it wakes as soon as the
+// phase completes), so waiting roles do not take issue slots from the warps
+// that share their scheduler.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -220,6 +226,54 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t (&a)[32], uint
         : "memory");
 }
 
+// 32 lanes x 64 consecutive columns in two x32 loads and one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+    uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : SIGATTN_R32(a), SIGATTN_R32(b)
+        : "r"(taddr), "r"(taddr + 32)
+        : "memory");
+}
+
+// 32 lanes x 128 consecutive columns in four x32 loads and one wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+    uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+    uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+    uint32_t(&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
+    uint32_t(&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : SIGATTN_R32(a), SIGATTN_R32(b), SIGATTN_R32(c), SIGATTN_R32(d)
+        : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+        : "memory");
+}
+
+// Two 64-column loads from different bases (e.g. S and dP) and one wait.
+__device__ __forceinline__ void tmem_ld64x2(uint32_t ta, uint32_t (&ra)[64], uint32_t tb,
+                                            uint32_t (&rb)[64]) {
+    uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&ra[0]);
+    uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&ra[32]);
+    uint32_t(&b0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&rb[0]);
+    uint32_t(&b1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&rb[32]);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : SIGATTN_R32(a0), SIGATTN_R32(a1), SIGATTN_R32(b0), SIGATTN_R32(b1)
+        : "r"(ta), "r"(ta + 32), "r"(tb), "r"(tb + 32)
+        : "memory");
+}
+
 // 32 lanes x 16 consecutive 32-bit columns, registers -> TMEM.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
@@ -231,6 +285,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+// 32 lanes x 32 consecutive 32-bit columns, registers -> TMEM.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -238,6 +306,16 @@ __device__ __forceinline__ void tmem_wait_st() {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Two finite floats to packed bf16 (lo in the low half),
+// rounding half away from zero: add half an ulp of bf16 to the bit pattern and
+// keep the high halves.  Differs from round-to-nearest-even only on exact
+// ties, and runs on the integer pipe instead of the conversion unit.
+__device__ __forceinline__ uint32_t pack_bf16x2_rh(float lo, float hi) {
+    const uint32_t a = __float_as_uint(lo) + 0x8000u;
+    const uint32_t b = __float_as_uint(hi) + 0x8000u;
+    return __byte_perm(a, b, 0x7632);
 }
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }

@@ -78,11 +78,18 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("mode", ["tanh", "exp"])
 @pytest.mark.parametrize("Z,L,H,D,nq,nk", SMALL)
-def test_bf16_small_full(Z, L, H, D, nq, nk):
+def test_bf16_small_full(Z, L, H, D, nq, nk, mode):
     dev = _dev()
     inp = _case(Z, L, H, D, nq, nk, seed=1000 + L + D)
-    _check_full(inp, _run(inp, dev), "bf16")
+    old = sa.get_sigmoid_mode()
+    sa.set_sigmoid_mode(sa.SIGMOID_TANH if mode == "tanh" else sa.SIGMOID_EXP)
+    try:
+        outs = _run(inp, dev)
+    finally:
+        sa.set_sigmoid_mode(old)
+    _check_full(inp, outs, "bf16")
 
 
 @pytest.mark.parametrize("Z,L,H,D,nq,nk", [(2, 128, 2, 64, (128, 77), (128, 77)),
@@ -122,15 +129,22 @@ def _check_sampled(inp, outs, per_sample, seed):
     return report
 
 
+@pytest.mark.parametrize("mode", ["tanh", "exp"])
 @pytest.mark.parametrize("index", [2, 3, 4, 5])
-def test_workload_sampled(index):
+def test_workload_sampled(index, mode):
+    """Full-size workloads, both in-register sigma forms, forward and backward."""
     dev = _dev()
     w = workloads.WORKLOADS[index]
     inp = workloads.make_inputs(w)
-    outs = _run(inp, dev)
+    old = sa.get_sigmoid_mode()
+    sa.set_sigmoid_mode(sa.SIGMOID_TANH if mode == "tanh" else sa.SIGMOID_EXP)
+    try:
+        outs = _run(inp, dev)
+    finally:
+        sa.set_sigmoid_mode(old)
     per = 48 if w.L >= 8192 else 96
     rep = _check_sampled(inp, outs, per, seed=index)
-    print(f"workload {index} ({w.name}):",
+    print(f"workload {index} ({w.name}), sigma {mode}: max-abs/max|ref| / L1 rel:",
           {k: ("%.2e/%.2e" % v) for k, v in rep.items()})
 
 
@@ -227,3 +241,4 @@ def test_autograd_module_matches_oracle():
     o.backward(g["dout"])
     torch.cuda.synchronize()
     _check_full(inp, (o.detach(), q.grad, k.grad, v.grad), "bf16")
+
