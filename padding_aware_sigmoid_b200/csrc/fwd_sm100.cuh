@@ -285,7 +285,6 @@ __global__ void __launch_bounds__(384, 1)
                     uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const int c = 64 * half + 2 * i;
                         const float2 pr = sigma2<MODE>(
                             scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
                         pk[i] = pack_bf16x2_rh(pr.x, pr.y);
