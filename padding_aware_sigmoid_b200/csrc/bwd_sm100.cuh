@@ -9,12 +9,15 @@
 // thread of warp 1 issues tcgen05.mma, and two warpgroups (warps 4-7 and
 // 8-11) turn the fp32 score tiles in TMEM into bf16 operands, each owning 64
 // of the 128 columns (thread = TMEM lane = tile row).  The bf16 results are
-// written back into TMEM over the columns their own warpgroup has already
-// read, and become the TMEM-resident A operand of the next MMA:
+// written back into TMEM over columns their own warpgroup has already read,
+// and become the TMEM-resident A operand of the next MMA:
 //   warpgroup 0 writes packed columns [base, base+32)     for tile columns 0..63
 //   warpgroup 1 writes packed columns [base+64, base+96)  for tile columns 64..127
 // so the MMA step kk (16 tile columns) reads TMEM column
 //   base + (kk < 4 ? 8 kk : 64 + 8 (kk - 4)).
+// The warpgroups hand their work over in two steps (first what depends on
+// the scores only, then what needs dP), so that the next scores' MMA runs
+// while the warpgroups still work on the current tile.
 #pragma once
 
 #include "fwd_sm100.cuh"
@@ -35,26 +38,55 @@ struct BwdParams {
     uint64_t timeout_ns;
 };
 
-template <int D, int STAGES>
+// Shared memory: two resident tiles (dq: Q, dO; dkdv: K, V) and two rings of
+// streamed tiles, X (dq: K_j; dkdv: Q_i) with SX slots and Y (dq: V_j; dkdv:
+// dO_i) with SY slots.  The rings are separate so that each tile's slot is
+// released as soon as its own last MMA has finished; X holds the tile whose
+// last use comes later in the step, so it gets the deeper ring.
+template <int D, int SX, int SY>
 struct BwdLayout {
     static constexpr int NSUB = D / 64;
     static constexpr int SUB_BYTES = 128 * 64 * 2;
     static constexpr int TILE_BYTES = NSUB * SUB_BYTES;
-    // two resident tiles (dq: Q, dO; dkdv: K, V) and a ring of streamed pairs
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = TILE_BYTES;
-    static constexpr int OFF_RING = 2 * TILE_BYTES;   // stage s: [X_s][Y_s]
-    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_RING + STAGES * STAGE_BYTES;
-    // res_full, ring_full[S], ring_empty[S], sdp_full, ds_full, mm_done, drain
-    static constexpr int NBAR = 1 + 2 * STAGES + 4;
+    static constexpr int OFF_X = 2 * TILE_BYTES;
+    static constexpr int OFF_Y = OFF_X + SX * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_Y + SY * TILE_BYTES;
+    // res_full, x_full[SX], x_empty[SX], y_full[SY], y_empty[SY], then up to
+    // MAX_HANDOFF per-kernel hand-off barriers
+    static constexpr int MAX_HANDOFF = 10;
+    static constexpr int NBAR = 1 + 2 * SX + 2 * SY + MAX_HANDOFF;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
     static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
     static_assert(COL_ACC1 + D <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
+
+// Streams tiles j = 0..n-1 of one tensor map into a ring of S slots; returns
+// false when a wait gave up.  `issued` counts the loads issued so far.
+template <int S, int NSUB>
+__device__ __forceinline__ bool ring_load(const CUtensorMap *map, uint64_t *full, uint64_t *empty,
+                                          uint8_t *base, int tile_bytes, int j, int h, int z,
+                                          const WaitCtx &w) {
+    const int st = j % S;
+    if (j >= S && !mbar_wait(&empty[st], ((j / S) - 1) & 1, w)) return false;
+    mbar_arrive_expect_tx(&full[st], tile_bytes);
+    for (int s = 0; s < NSUB; ++s)
+        tma_load_4d(map, &full[st], base + st * tile_bytes + s * (128 * 64 * 2), 64 * s, h, j * 128, z);
+    return true;
+}
+
+// Waits (time-bounded, ignoring the abort flag) until the last min(issued, S)
+// loads of a ring have landed, so no TMA write is in flight at exit.
+template <int S>
+__device__ __forceinline__ void ring_drain(uint64_t *full, int issued, uint64_t limit_ns) {
+    for (int j = (issued > S ? issued - S : 0); j < issued; ++j)
+        mbar_wait_drain(&full[j % S], (j / S) & 1, limit_ns);
+}
 
 __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
 
@@ -87,26 +119,56 @@ __device__ __forceinline__ void zero_row(__nv_bfloat16 *dst, int col0, int ncols
     for (int v4 = 0; v4 < ncols / 8; ++v4) o[v4] = make_uint4(0u, 0u, 0u, 0u);
 }
 
+// Packs 32 pairs to bf16 and zeroes the entries at tile columns >= valid
+// (columns [col0, col0 + 64) of the tile; valid = count of in-range columns).
+__device__ __forceinline__ void mask_packed(uint32_t (&pk)[32], int col0, int valid) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int c = col0 + 2 * i;
+        const uint32_t lo = c < valid ? 0x0000FFFFu : 0u;
+        const uint32_t hi = c + 1 < valid ? 0xFFFF0000u : 0u;
+        pk[i] &= (lo | hi);
+    }
+}
+
 // ============================================================================
 // dQ kernel: one CTA per 128-row query tile; streams K_j, V_j for j < ceil(n_k/128).
-// TMEM: [0,128) S -> dS (bf16, packed), [128,256) dP, [256,256+D) dQ.
+// TMEM: [0,128) S, [128,256) and [256,384) dP of even / odd key tiles (each
+// overwritten by its dS, bf16 packed), [384,384+D) dQ.
+//
+// Per key tile j the warpgroups (1) read S_j and release it, keeping
+// sigma'(S_j) in registers, then (2) read dP_j and write dS_j = sigma' dP_j
+// over dP_j.  The MMA thread issues S_{j+1} as soon as S_j is released and
+// dP_{j+1} into the other dP buffer (free once dQ += dS_{j-1} K_{j-1} has
+// finished), then dQ += dS_j K_j when dS_j is ready: neither warpgroup phase
+// waits on the MMA that consumes the previous tile.  The two warpgroups take
+// turns for the sigma' phase (warpgroup 0 first), so that it has the MUFU to
+// itself while the other warpgroup forms dS.
 // ============================================================================
-template <int D, int MODE, int STAGES>
+template <int D, int MODE, int SX, int SY>
 __global__ void __launch_bounds__(384, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BwdParams p) {
-    using Lay = BwdLayout<D, STAGES>;
+    using Lay = BwdLayout<D, SX, SY>;
+    constexpr uint32_t kColS = 0, kColDP0 = 128, kColDP1 = 256, kColDQ = 384;
+    static_assert(kColDQ + D <= Lay::TMEM_COLS, "TMEM budget");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::OFF_BAR);
     uint64_t *res_full = bars;
-    uint64_t *ring_full = bars + 1;
-    uint64_t *ring_empty = ring_full + STAGES;
-    uint64_t *sdp_full = ring_empty + STAGES;
-    uint64_t *ds_full = sdp_full + 1;
-    uint64_t *mm_done = ds_full + 1;
-    uint64_t *drain = mm_done + 1;
+    uint64_t *x_full = bars + 1;              // K_j ring
+    uint64_t *x_empty = x_full + SX;
+    uint64_t *y_full = x_empty + SX;          // V_j ring
+    uint64_t *y_empty = y_full + SY;
+    uint64_t *s_full = y_empty + SY;          // MMA -> WGs: S_j in TMEM
+    uint64_t *dp_full = s_full + 1;           // [2] MMA -> WGs: dP_j in buffer j % 2
+    uint64_t *s_free = dp_full + 2;           // WGs -> MMA: S_j read
+    uint64_t *ds_ready = s_free + 1;          // [2] WGs -> MMA: dS_j in buffer j % 2
+    uint64_t *dq_done = ds_ready + 2;         // MMA -> all: dQ += dS_j K_j finished
+    uint64_t *drain = dq_done + 1;
+    uint64_t *turn = drain + 1;               // [2] sigma' phase token per warpgroup
+    static_assert(10 <= Lay::MAX_HANDOFF, "barrier count");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -124,14 +186,24 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(res_full, 1);
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&ring_full[s], 1);
-            mbar_init(&ring_empty[s], 1);
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1);
         }
-        mbar_init(sdp_full, 1);
-        mbar_init(ds_full, 256);
-        mbar_init(mm_done, 1);
+        for (int s = 0; s < SY; ++s) {
+            mbar_init(&y_full[s], 1);
+            mbar_init(&y_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(&dp_full[0], 1);
+        mbar_init(&dp_full[1], 1);
+        mbar_init(s_free, 256);
+        mbar_init(&ds_ready[0], 256);
+        mbar_init(&ds_ready[1], 256);
+        mbar_init(dq_done, 1);
         mbar_init(drain, 1);
+        mbar_init(&turn[0], 128);
+        mbar_init(&turn[1], 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -153,64 +225,84 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp == 0) {
         if (work && lane == 0) {
-            uint8_t *sQ = smem + Lay::OFF_A, *sDO = smem + Lay::OFF_B, *ring = smem + Lay::OFF_RING;
+            uint8_t *sQ = smem + Lay::OFF_A, *sDO = smem + Lay::OFF_B;
             mbar_arrive_expect_tx(res_full, 2 * Lay::TILE_BYTES);
             for (int s = 0; s < Lay::NSUB; ++s) {
                 tma_load_4d(&tmQ, res_full, sQ + s * Lay::SUB_BYTES, 64 * s, h, qtile * 128, z);
                 tma_load_4d(&tmDO, res_full, sDO + s * Lay::SUB_BYTES, 64 * s, h, qtile * 128, z);
             }
-            int issued = 0;
+            int ix = 0, iy = 0;
             for (int j = 0; j < nkv; ++j) {
-                const int st = j % STAGES, round = j / STAGES;
-                if (j >= STAGES && !mbar_wait(&ring_empty[st], (round - 1) & 1, wctx)) break;
-                uint8_t *sK = ring + st * Lay::STAGE_BYTES, *sV = sK + Lay::TILE_BYTES;
-                mbar_arrive_expect_tx(&ring_full[st], 2 * Lay::TILE_BYTES);
-                for (int s = 0; s < Lay::NSUB; ++s) {
-                    tma_load_4d(&tmK, &ring_full[st], sK + s * Lay::SUB_BYTES, 64 * s, h, j * 128, z);
-                    tma_load_4d(&tmV, &ring_full[st], sV + s * Lay::SUB_BYTES, 64 * s, h, j * 128, z);
-                }
-                issued = j + 1;
+                if (!ring_load<SX, Lay::NSUB>(&tmK, x_full, x_empty, smem + Lay::OFF_X, Lay::TILE_BYTES,
+                                             j, h, z, wctx))
+                    break;
+                ix = j + 1;
+                if (!ring_load<SY, Lay::NSUB>(&tmV, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
+                                             j, h, z, wctx))
+                    break;
+                iy = j + 1;
             }
             mbar_wait_drain(res_full, 0, p.timeout_ns);
-            for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-                mbar_wait_drain(&ring_full[j % STAGES], (j / STAGES) & 1, p.timeout_ns);
+            ring_drain<SX>(x_full, ix, p.timeout_ns);
+            ring_drain<SY>(y_full, iy, p.timeout_ns);
         }
     } else if (warp == 1) {
         if (work && lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idesc_q = idesc_bf16_f32(128, D, false, true);
             const uint32_t sQ = smem_u32(smem + Lay::OFF_A), sDO = smem_u32(smem + Lay::OFF_B);
-            const uint32_t ring = smem_u32(smem + Lay::OFF_RING);
-            bool ok = mbar_wait(res_full, 0, wctx);
+            const uint32_t xring = smem_u32(smem + Lay::OFF_X), yring = smem_u32(smem + Lay::OFF_Y);
+            auto kslot = [&](int j) { return xring + (j % SX) * Lay::TILE_BYTES; };
+            auto vslot = [&](int j) { return yring + (j % SY) * Lay::TILE_BYTES; };
+            // X (128 rows of Q or dO) times Y^T (128 rows of K or V) into TMEM column `col`
+            auto issue_xyT = [&](uint32_t col, uint32_t xbase, uint32_t ybase) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
+                    mma_ss(tmem + col, smem_desc_sw128(xbase + koff, 16, 1024),
+                           smem_desc_sw128(ybase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(res_full, 0, wctx) && mbar_wait(&x_full[0], 0, wctx) &&
+                      mbar_wait(&y_full[0], 0, wctx);
+            if (ok) {
+                tc_fence_after();
+                issue_xyT(kColS, sQ, kslot(0));
+                mma_commit(s_full);
+                issue_xyT(kColDP0, sDO, vslot(0));
+                mma_commit(&dp_full[0]);
+                mma_commit(&y_empty[0]);
+            }
             for (int j = 0; ok && j < nkv; ++j) {
-                const int st = j % STAGES, round = j / STAGES;
-                if (!(ok = mbar_wait(&ring_full[st], round & 1, wctx))) break;
-                if (j > 0 && !(ok = mbar_wait(mm_done, (j - 1) & 1, wctx))) break;
-                tc_fence_after();
-                const uint32_t sK = ring + st * Lay::STAGE_BYTES, sV = sK + Lay::TILE_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + Lay::COL_S, smem_desc_sw128(sQ + koff, 16, 1024),
-                           smem_desc_sw128(sK + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                const bool more = j + 1 < nkv;
+                if (more) {
+                    if (!(ok = mbar_wait(&x_full[(j + 1) % SX], ((j + 1) / SX) & 1, wctx))) break;
+                    if (!(ok = mbar_wait(s_free, j & 1, wctx))) break;
+                    trace(1, j, 0);
+                    tc_fence_after();
+                    issue_xyT(kColS, sQ, kslot(j + 1));
+                    mma_commit(s_full);
+                    if (!(ok = mbar_wait(&y_full[(j + 1) % SY], ((j + 1) / SY) & 1, wctx))) break;
+                    // buffer (j+1) % 2 holds dS_{j-1} until dQ += dS_{j-1} K_{j-1} is done
+                    if (j > 0 && !(ok = mbar_wait(dq_done, (j - 1) & 1, wctx))) break;
+                    trace(1, j, 1);
+                    tc_fence_after();
+                    issue_xyT((j + 1) & 1 ? kColDP1 : kColDP0, sDO, vslot(j + 1));
+                    mma_commit(&dp_full[(j + 1) & 1]);
+                    mma_commit(&y_empty[(j + 1) % SY]);   // V_{j+1}: its only MMA
                 }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + Lay::COL_DP, smem_desc_sw128(sDO + koff, 16, 1024),
-                           smem_desc_sw128(sV + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(sdp_full);
-                if (!(ok = mbar_wait(ds_full, j & 1, wctx))) break;
+                if (!(ok = mbar_wait(&ds_ready[j & 1], (j >> 1) & 1, wctx))) break;
+                trace(1, j, 2);
                 tc_fence_after();
+                const uint32_t dcol = j & 1 ? kColDP1 : kColDP0;
+                const uint32_t sK = kslot(j);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_ts(tmem + Lay::COL_ACC0, tmem + Lay::COL_S + packed_col(kk),
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + kColDQ, tmem + dcol + packed_col(kk),
                            smem_desc_sw128(sK + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_q,
                            (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(mm_done);
-                mma_commit(&ring_empty[st]);
+                mma_commit(dq_done);
+                mma_commit(&x_empty[j % SX]);             // K_j: S_j and dQ_j done
             }
             mma_commit(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
@@ -226,42 +318,58 @@ __global__ void __launch_bounds__(384, 1)
         if (work) {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
             for (int j = 0; j < nkv; ++j) {
-                ok = __all_sync(0xffffffffu, mbar_wait(sdp_full, j & 1, wctx));
-                if (!ok) break;
-                tc_fence_after();
-                const int kbase = j * 128;
-                const bool partial = kbase + 128 > nk;
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int col = 64 * w + 32 * c;
-                    uint32_t rs[32], rd[32];
-                    tmem_ld32x2(tmem + lane_bits + Lay::COL_S + col, rs,
-                                tmem + lane_bits + Lay::COL_DP + col, rd);
-                                        uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float2 pr, gr;
-                        sigma_grad2<MODE>(scale2(__uint_as_float(rs[2 * i]), __uint_as_float(rs[2 * i + 1]), cf),
-                                          pr, gr);
-                        const float2 ds = mul2(gr, f2(__uint_as_float(rd[2 * i]), __uint_as_float(rd[2 * i + 1])));
-                        float ds0 = ds.x, ds1 = ds.y;
-                        if (partial) {
-                            const int key = kbase + col + 2 * i;
-                            if (key >= nk) ds0 = 0.0f;
-                            if (key + 1 >= nk) ds1 = 0.0f;
-                        }
-                        pk[i] = pack_bf16x2(ds0, ds1);
+                float2 g[32];
+                {
+                    if (quarter == 0) trace(2 + w, j, 0);
+                    ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, wctx));
+                    if (!ok) break;
+                    if (quarter == 0) trace(2 + w, j, 1);
+                    tc_fence_after();
+                    uint32_t r[64];
+                    tmem_ld64(tmem + lane_bits + kColS + 64 * w, r);
+                    if (quarter == 0) trace(2 + w, j, 2);
+                    tc_fence_before();
+                    mbar_arrive(s_free);
+                    if (w == 1 || j > 0) {
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait(&turn[w], (w == 0 ? j - 1 : j) & 1, wctx));
+                        if (!ok) break;
                     }
-                    tmem_st16(tmem + lane_bits + Lay::COL_S + 64 * w + 16 * c, pk);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float2 pr;
+                        sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf),
+                                          pr, g[i]);
+                    }
+                    mbar_arrive(&turn[w ^ 1]);
                 }
+                const uint32_t dcol = (j & 1 ? kColDP1 : kColDP0) + 64 * w;
+                if (quarter == 0) trace(2 + w, j, 3);
+                ok = __all_sync(0xffffffffu, mbar_wait(&dp_full[j & 1], (j >> 1) & 1, wctx));
+                if (!ok) break;
+                if (quarter == 0) trace(2 + w, j, 4);
+                tc_fence_after();
+                uint32_t d[64];
+                tmem_ld64(tmem + lane_bits + dcol, d);
+                if (quarter == 0) trace(2 + w, j, 5);
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float2 ds = mul2(g[i], f2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
+                    pk[i] = pack_bf16x2(ds.x, ds.y);
+                }
+                const int kvalid = nk - j * 128;
+                if (kvalid < 128) mask_packed(pk, 64 * w, kvalid);
+                tmem_st32(tmem + lane_bits + dcol, pk);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(ds_full);
+                mbar_arrive(&ds_ready[j & 1]);
+                if (quarter == 0) trace(2 + w, j, 6);
             }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(mm_done, (nkv - 1) & 1, wctx));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dq_done, (nkv - 1) & 1, wctx));
             if (ok) {
                 tc_fence_after();
-                store_row_from_tmem<D>(tmem + lane_bits + Lay::COL_ACC0, drow, row < L, row < nq,
+                store_row_from_tmem<D>(tmem + lane_bits + kColDQ, drow, row < L, row < nq,
                                        p.alpha, w * (D / 2), D / 2);
             }
         } else if (row < L) {
@@ -283,23 +391,34 @@ __global__ void __launch_bounds__(384, 1)
 //   S^T = K Q_i^T, dP^T = V dO_i^T, P^T -> TMEM over S^T, dS^T -> TMEM over dP^T,
 //   dV += P^T dO_i, dK += dS^T Q_i.
 // TMEM: [0,128) S^T / P^T, [128,256) dP^T / dS^T, [256,256+D) dV, [256+D,256+2D) dK.
+//
+// The warpgroups publish P^T first (it needs S^T only) and dS^T second; the
+// MMA order per query tile is dV_i, S^T_{i+1} (after dV_i consumed P^T_i),
+// dK_i, dP^T_{i+1} (after dK_i consumed dS^T_i), so the sigma work on i+1
+// overlaps dK_i.
 // ============================================================================
-template <int D, int MODE, int STAGES>
+template <int D, int MODE, int SX, int SY>
 __global__ void __launch_bounds__(384, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const BwdParams p) {
-    using Lay = BwdLayout<D, STAGES>;
+    using Lay = BwdLayout<D, SX, SY>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::OFF_BAR);
     uint64_t *res_full = bars;
-    uint64_t *ring_full = bars + 1;
-    uint64_t *ring_empty = ring_full + STAGES;
-    uint64_t *sdp_full = ring_empty + STAGES;
-    uint64_t *pds_full = sdp_full + 1;
-    uint64_t *mm_done = pds_full + 1;
-    uint64_t *drain = mm_done + 1;
+    uint64_t *x_full = bars + 1;              // Q_i ring
+    uint64_t *x_empty = x_full + SX;
+    uint64_t *y_full = x_empty + SX;          // dO_i ring
+    uint64_t *y_empty = y_full + SY;
+    uint64_t *s_full = y_empty + SY;          // MMA -> WGs: S^T_i in TMEM
+    uint64_t *dp_full = s_full + 1;           // MMA -> WGs: dP^T_i in TMEM
+    uint64_t *p_ready = dp_full + 1;          // WGs -> MMA: P^T_i in TMEM
+    uint64_t *ds_ready = p_ready + 1;         // WGs -> MMA: dS^T_i in TMEM
+    uint64_t *dv_done = ds_ready + 1;         // MMA: dV += P^T_i dO_i finished
+    uint64_t *dk_done = dv_done + 1;          // MMA: dK += dS^T_i Q_i finished
+    uint64_t *drain = dk_done + 1;
+    static_assert(7 <= Lay::MAX_HANDOFF, "barrier count");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -317,13 +436,20 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(res_full, 1);
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&ring_full[s], 1);
-            mbar_init(&ring_empty[s], 1);
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1);
         }
-        mbar_init(sdp_full, 1);
-        mbar_init(pds_full, 256);
-        mbar_init(mm_done, 1);
+        for (int s = 0; s < SY; ++s) {
+            mbar_init(&y_full[s], 1);
+            mbar_init(&y_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(dp_full, 1);
+        mbar_init(p_ready, 256);
+        mbar_init(ds_ready, 256);
+        mbar_init(dv_done, 1);
+        mbar_init(dk_done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -346,70 +472,86 @@ __global__ void __launch_bounds__(384, 1)
 
     if (warp == 0) {
         if (work && lane == 0) {
-            uint8_t *sK = smem + Lay::OFF_A, *sV = smem + Lay::OFF_B, *ring = smem + Lay::OFF_RING;
+            uint8_t *sK = smem + Lay::OFF_A, *sV = smem + Lay::OFF_B;
             mbar_arrive_expect_tx(res_full, 2 * Lay::TILE_BYTES);
             for (int s = 0; s < Lay::NSUB; ++s) {
                 tma_load_4d(&tmK, res_full, sK + s * Lay::SUB_BYTES, 64 * s, h, ktile * 128, z);
                 tma_load_4d(&tmV, res_full, sV + s * Lay::SUB_BYTES, 64 * s, h, ktile * 128, z);
             }
-            int issued = 0;
+            int ix = 0, iy = 0;
             for (int i = 0; i < nqt; ++i) {
-                const int st = i % STAGES, round = i / STAGES;
-                if (i >= STAGES && !mbar_wait(&ring_empty[st], (round - 1) & 1, wctx)) break;
-                uint8_t *sQ = ring + st * Lay::STAGE_BYTES, *sDO = sQ + Lay::TILE_BYTES;
-                mbar_arrive_expect_tx(&ring_full[st], 2 * Lay::TILE_BYTES);
-                for (int s = 0; s < Lay::NSUB; ++s) {
-                    tma_load_4d(&tmQ, &ring_full[st], sQ + s * Lay::SUB_BYTES, 64 * s, h, i * 128, z);
-                    tma_load_4d(&tmDO, &ring_full[st], sDO + s * Lay::SUB_BYTES, 64 * s, h, i * 128, z);
-                }
-                issued = i + 1;
+                if (!ring_load<SX, Lay::NSUB>(&tmQ, x_full, x_empty, smem + Lay::OFF_X, Lay::TILE_BYTES,
+                                             i, h, z, wctx))
+                    break;
+                ix = i + 1;
+                if (!ring_load<SY, Lay::NSUB>(&tmDO, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
+                                             i, h, z, wctx))
+                    break;
+                iy = i + 1;
             }
             mbar_wait_drain(res_full, 0, p.timeout_ns);
-            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-                mbar_wait_drain(&ring_full[i % STAGES], (i / STAGES) & 1, p.timeout_ns);
+            ring_drain<SX>(x_full, ix, p.timeout_ns);
+            ring_drain<SY>(y_full, iy, p.timeout_ns);
         }
     } else if (warp == 1) {
         if (work && lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);
             const uint32_t sK = smem_u32(smem + Lay::OFF_A), sV = smem_u32(smem + Lay::OFF_B);
-            const uint32_t ring = smem_u32(smem + Lay::OFF_RING);
-            bool ok = mbar_wait(res_full, 0, wctx);
+            const uint32_t xring = smem_u32(smem + Lay::OFF_X), yring = smem_u32(smem + Lay::OFF_Y);
+            auto qslot = [&](int i) { return xring + (i % SX) * Lay::TILE_BYTES; };
+            auto doslot = [&](int i) { return yring + (i % SY) * Lay::TILE_BYTES; };
+            auto issue_xyT = [&](uint32_t col, uint32_t xbase, uint32_t ybase) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
+                    mma_ss(tmem + col, smem_desc_sw128(xbase + koff, 16, 1024),
+                           smem_desc_sw128(ybase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+            };
+            // acc += A(TMEM, packed over `acol`) * B (128 query rows, MN-major)
+            auto issue_acc = [&](uint32_t acc, uint32_t acol, uint32_t bbase, bool first) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + acc, tmem + acol + packed_col(kk),
+                           smem_desc_sw128(bbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_kv,
+                           (!first || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(res_full, 0, wctx) && mbar_wait(&x_full[0], 0, wctx) &&
+                      mbar_wait(&y_full[0], 0, wctx);
+            if (ok) {
+                tc_fence_after();
+                issue_xyT(Lay::COL_S, sK, qslot(0));
+                mma_commit(s_full);
+                issue_xyT(Lay::COL_DP, sV, doslot(0));
+                mma_commit(dp_full);
+            }
             for (int i = 0; ok && i < nqt; ++i) {
-                const int st = i % STAGES, round = i / STAGES;
-                if (!(ok = mbar_wait(&ring_full[st], round & 1, wctx))) break;
-                if (i > 0 && !(ok = mbar_wait(mm_done, (i - 1) & 1, wctx))) break;
+                const bool more = i + 1 < nqt;
+                if (!(ok = mbar_wait(p_ready, i & 1, wctx))) break;
                 tc_fence_after();
-                const uint32_t sQ = ring + st * Lay::STAGE_BYTES, sDO = sQ + Lay::TILE_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + Lay::COL_S, smem_desc_sw128(sK + koff, 16, 1024),
-                           smem_desc_sw128(sQ + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                issue_acc(Lay::COL_ACC0, Lay::COL_S, doslot(i), i == 0);      // dV += P^T dO_i
+                mma_commit(dv_done);
+                mma_commit(&y_empty[i % SY]);                                 // dO_i: dP^T_i, dV_i done
+                if (more) {
+                    if (!(ok = mbar_wait(&x_full[(i + 1) % SX], ((i + 1) / SX) & 1, wctx))) break;
+                    if (!(ok = mbar_wait(dv_done, i & 1, wctx))) break;   // P^T_i consumed
+                    tc_fence_after();
+                    issue_xyT(Lay::COL_S, sK, qslot(i + 1));
+                    mma_commit(s_full);
                 }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + Lay::COL_DP, smem_desc_sw128(sV + koff, 16, 1024),
-                           smem_desc_sw128(sDO + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(sdp_full);
-                if (!(ok = mbar_wait(pds_full, i & 1, wctx))) break;
+                if (!(ok = mbar_wait(ds_ready, i & 1, wctx))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_ts(tmem + Lay::COL_ACC0, tmem + Lay::COL_S + packed_col(kk),
-                           smem_desc_sw128(sDO + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_kv,
-                           (i > 0 || kk > 0) ? 1u : 0u);
+                issue_acc(Lay::COL_ACC1, Lay::COL_DP, qslot(i), i == 0);      // dK += dS^T Q_i
+                mma_commit(dk_done);
+                mma_commit(&x_empty[i % SX]);                                 // Q_i: S^T_i, dK_i done
+                if (more) {
+                    if (!(ok = mbar_wait(&y_full[(i + 1) % SY], ((i + 1) / SY) & 1, wctx))) break;
+                    if (!(ok = mbar_wait(dk_done, i & 1, wctx))) break;   // dS^T_i consumed
+                    tc_fence_after();
+                    issue_xyT(Lay::COL_DP, sV, doslot(i + 1));
+                    mma_commit(dp_full);
                 }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_ts(tmem + Lay::COL_ACC1, tmem + Lay::COL_DP + packed_col(kk),
-                           smem_desc_sw128(sQ + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_kv,
-                           (i > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(mm_done);
-                mma_commit(&ring_empty[st]);
             }
             mma_commit(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
@@ -426,41 +568,48 @@ __global__ void __launch_bounds__(384, 1)
         if (work) {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
             for (int i = 0; i < nqt; ++i) {
-                ok = __all_sync(0xffffffffu, mbar_wait(sdp_full, i & 1, wctx));
+                const int qvalid = nq - i * 128;
+                float2 g[32];
+                {
+                    ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
+                    if (!ok) break;
+                    tc_fence_after();
+                    uint32_t r[64];
+                    tmem_ld64(tmem + lane_bits + Lay::COL_S + 64 * w, r);
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int ii = 0; ii < 32; ++ii) {
+                        float2 pr;
+                        sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * ii]), __uint_as_float(r[2 * ii + 1]), cf),
+                                          pr, g[ii]);
+                        pk[ii] = pack_bf16x2(pr.x, pr.y);
+                    }
+                    if (qvalid < 128) mask_packed(pk, 64 * w, qvalid);
+                    tmem_st32(tmem + lane_bits + Lay::COL_S + 64 * w, pk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(p_ready);
+                }
+                ok = __all_sync(0xffffffffu, mbar_wait(dp_full, i & 1, wctx));
                 if (!ok) break;
                 tc_fence_after();
-                const int qbase = i * 128;
-                const bool partial = qbase + 128 > nq;
+                uint32_t d[64];
+                tmem_ld64(tmem + lane_bits + Lay::COL_DP + 64 * w, d);
+                uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int col = 64 * w + 32 * c;
-                    uint32_t rs[32], rd[32];
-                    tmem_ld32x2(tmem + lane_bits + Lay::COL_S + col, rs,
-                                tmem + lane_bits + Lay::COL_DP + col, rd);
-                                        uint32_t pkp[16], pks[16];
-#pragma unroll
-                    for (int ii = 0; ii < 16; ++ii) {
-                        float2 pr, gr;
-                        sigma_grad2<MODE>(scale2(__uint_as_float(rs[2 * ii]), __uint_as_float(rs[2 * ii + 1]), cf),
-                                          pr, gr);
-                        const float2 ds = mul2(gr, f2(__uint_as_float(rd[2 * ii]), __uint_as_float(rd[2 * ii + 1])));
-                        float p0 = pr.x, p1 = pr.y, ds0 = ds.x, ds1 = ds.y;
-                        if (partial) {
-                            const int q = qbase + col + 2 * ii;
-                            if (q >= nq) { p0 = 0.0f; ds0 = 0.0f; }
-                            if (q + 1 >= nq) { p1 = 0.0f; ds1 = 0.0f; }
-                        }
-                        pkp[ii] = pack_bf16x2(p0, p1);
-                        pks[ii] = pack_bf16x2(ds0, ds1);
-                    }
-                    tmem_st16(tmem + lane_bits + Lay::COL_S + 64 * w + 16 * c, pkp);
-                    tmem_st16(tmem + lane_bits + Lay::COL_DP + 64 * w + 16 * c, pks);
+                for (int ii = 0; ii < 32; ++ii) {
+                    const float2 ds = mul2(g[ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
+                    pk[ii] = pack_bf16x2(ds.x, ds.y);
                 }
+                if (qvalid < 128) mask_packed(pk, 64 * w, qvalid);
+                tmem_st32(tmem + lane_bits + Lay::COL_DP + 64 * w, pk);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(pds_full);
+                mbar_arrive(ds_ready);
             }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(mm_done, (nqt - 1) & 1, wctx));
+            if (ok)
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(w == 0 ? dv_done : dk_done, (nqt - 1) & 1, wctx));
             if (ok) {
                 tc_fence_after();
                 store_row_from_tmem<D>(tmem + lane_bits + (w == 0 ? Lay::COL_ACC0 : Lay::COL_ACC1), dst,

@@ -39,7 +39,10 @@ struct FwdParams {
     uint64_t timeout_ns;
 };
 
-template <int D, int STAGES>
+// Shared memory: the two query tiles, a ring of KS key tiles and a ring of VS
+// value tiles (V_j's last use, O += P V_j, comes later than K_j's, so its ring
+// is the deeper one).
+template <int D, int KS, int VS>
 struct FwdLayout {
     static constexpr int BM = 128;                 // query rows per tile
     static constexpr int BN = 128;                 // keys per tile
@@ -48,11 +51,11 @@ struct FwdLayout {
     static constexpr int TILE_BYTES = NSUB * SUB_BYTES;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
-    static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_V + STAGES * TILE_BYTES;
-    // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
+    static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
+    // q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2],
     // pv_done[2], drain, turn[2]
-    static constexpr int NBAR = 1 + 4 * STAGES + 9;
+    static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 9;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
     static constexpr int BYTES = OFF_ABORT + 8;
@@ -60,6 +63,7 @@ struct FwdLayout {
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
     static_assert(COL_O1 + D <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ uint8_t *align_1k(uint8_t *p) {
@@ -77,24 +81,25 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, 
     }
 }
 
-template <int D, int MODE, int STAGES>
+template <int D, int MODE, int KS, int VS>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-    using Lay = FwdLayout<D, STAGES>;
+    using Lay = FwdLayout<D, KS, VS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::OFF_BAR);
     uint64_t *q_full = bars;
     uint64_t *k_full = bars + 1;
-    uint64_t *k_empty = k_full + STAGES;
-    uint64_t *v_full = k_empty + STAGES;
-    uint64_t *v_empty = v_full + STAGES;
-    uint64_t *s_full = v_empty + STAGES;
+    uint64_t *k_empty = k_full + KS;
+    uint64_t *v_full = k_empty + KS;
+    uint64_t *v_empty = v_full + VS;
+    uint64_t *s_full = v_empty + VS;
     uint64_t *p_full = s_full + 2;
     uint64_t *pv_done = p_full + 2;
     uint64_t *drain = pv_done + 2;
     uint64_t *turn = drain + 1;
+    static_assert(1 + 2 * KS + 2 * VS + 9 == Lay::NBAR, "barrier count");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -115,9 +120,11 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < KS; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < VS; ++s) {
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
@@ -160,26 +167,26 @@ __global__ void __launch_bounds__(384, 1)
                                 64 * s, h, (qtile0 + t) * Lay::BM, z);
             int issued_k = 0, issued_v = 0;
             for (int j = 0; j < nkv; ++j) {
-                const int st = j % STAGES, round = j / STAGES;
-                if (j >= STAGES && !mbar_wait(&k_empty[st], (round - 1) & 1, wctx)) break;
-                mbar_arrive_expect_tx(&k_full[st], Lay::TILE_BYTES);
+                const int sk = j % KS, sv = j % VS;
+                if (j >= KS && !mbar_wait(&k_empty[sk], ((j / KS) - 1) & 1, wctx)) break;
+                mbar_arrive_expect_tx(&k_full[sk], Lay::TILE_BYTES);
                 for (int s = 0; s < Lay::NSUB; ++s)
-                    tma_load_4d(&tmK, &k_full[st], sK + st * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
+                    tma_load_4d(&tmK, &k_full[sk], sK + sk * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
                                 64 * s, h, j * Lay::BN, z);
                 issued_k = j + 1;
-                if (j >= STAGES && !mbar_wait(&v_empty[st], (round - 1) & 1, wctx)) break;
-                mbar_arrive_expect_tx(&v_full[st], Lay::TILE_BYTES);
+                if (j >= VS && !mbar_wait(&v_empty[sv], ((j / VS) - 1) & 1, wctx)) break;
+                mbar_arrive_expect_tx(&v_full[sv], Lay::TILE_BYTES);
                 for (int s = 0; s < Lay::NSUB; ++s)
-                    tma_load_4d(&tmV, &v_full[st], sV + st * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
+                    tma_load_4d(&tmV, &v_full[sv], sV + sv * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
                                 64 * s, h, j * Lay::BN, z);
                 issued_v = j + 1;
             }
             // Every issued load must land before the CTA's shared memory is released.
             mbar_wait_drain(q_full, 0, p.timeout_ns);
-            for (int j = (issued_k > STAGES ? issued_k - STAGES : 0); j < issued_k; ++j)
-                mbar_wait_drain(&k_full[j % STAGES], (j / STAGES) & 1, p.timeout_ns);
-            for (int j = (issued_v > STAGES ? issued_v - STAGES : 0); j < issued_v; ++j)
-                mbar_wait_drain(&v_full[j % STAGES], (j / STAGES) & 1, p.timeout_ns);
+            for (int j = (issued_k > KS ? issued_k - KS : 0); j < issued_k; ++j)
+                mbar_wait_drain(&k_full[j % KS], (j / KS) & 1, p.timeout_ns);
+            for (int j = (issued_v > VS ? issued_v - VS : 0); j < issued_v; ++j)
+                mbar_wait_drain(&v_full[j % VS], (j / VS) & 1, p.timeout_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -223,19 +230,19 @@ __global__ void __launch_bounds__(384, 1)
                 mma_commit(&k_empty[0]);
             }
             for (int j = 0; ok && j < nkv; ++j) {
-                const int stv = j % STAGES;
-                const int stk = (j + 1) % STAGES;
+                const int stv = j % VS;
+                const int stk = (j + 1) % KS;
                 const bool more = j + 1 < nkv;
                 const uint32_t vbase = sV + stv * Lay::TILE_BYTES;
                 const uint32_t knext = sK + stk * Lay::TILE_BYTES;
-                if (!(ok = mbar_wait(&v_full[stv], (j / STAGES) & 1, wctx))) break;
+                if (!(ok = mbar_wait(&v_full[stv], (j / VS) & 1, wctx))) break;
                 for (int t = 0; t < ntiles; ++t) {
                     if (!(ok = mbar_wait(&p_full[t], j & 1, wctx))) break;
                     tc_fence_after();
                     issue_pv(t, vbase, j == 0);
                     if (t == ntiles - 1) mma_commit(&v_empty[stv]);
                     if (more) {
-                        if (t == 0 && !(ok = mbar_wait(&k_full[stk], ((j + 1) / STAGES) & 1, wctx))) break;
+                        if (t == 0 && !(ok = mbar_wait(&k_full[stk], ((j + 1) / KS) & 1, wctx))) break;
                         if (!(ok = mbar_wait(&pv_done[t], j & 1, wctx))) break;
                         tc_fence_after();
                         issue_s(t, knext);
@@ -287,7 +294,11 @@ __global__ void __launch_bounds__(384, 1)
                     for (int i = 0; i < 32; ++i) {
                         const float2 pr = sigma2<MODE>(
                             scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
+#ifdef SIGATTN_FWD_PACK_CVT
+                        pk[i] = pack_bf16x2(pr.x, pr.y);
+#else
                         pk[i] = pack_bf16x2_rh(pr.x, pr.y);
+#endif
                     }
                     if (kvalid < Lay::BN) {
                         // last tile: keys at or beyond n_k weigh exactly zero

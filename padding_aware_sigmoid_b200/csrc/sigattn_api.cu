@@ -18,9 +18,10 @@ namespace {
 using namespace sigattn;
 
 constexpr int kMaxDevices = 64;
-constexpr int kFwdStagesD128 = 2;
-constexpr int kFwdStagesD64 = 4;
-constexpr int kBwdStages = 2;
+// forward rings: key and value slots per head dim
+template <int D> struct FwdStages { static constexpr int K = D == 128 ? 2 : 4, V = D == 128 ? 3 : 4; };
+// backward rings: X (dq: K, dkdv: Q) and Y (dq: V, dkdv: dO) slots per head dim
+template <int D> struct BwdStages { static constexpr int X = D == 128 ? 3 : 4, Y = D == 128 ? 2 : 4; };
 
 std::mutex g_mu;
 int *g_status[kMaxDevices] = {};          // device status word per device (lazy, never freed)
@@ -130,10 +131,10 @@ sigattn_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 template <int D, int MODE>
 sigattn_status fwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                         const FwdParams &p, int Z, int L, int H, cudaStream_t st) {
-    constexpr int S = D == 128 ? kFwdStagesD128 : kFwdStagesD64;
+    constexpr int KS = FwdStages<D>::K, VS = FwdStages<D>::V;
     dim3 grid((L + 255) / 256, H, Z);
-    return launch(fwd_kernel<D, MODE, S>, grid, dim3(384), FwdLayout<D, S>::SMEM_ALLOC, st, mq, mk,
-                  mv, p);
+    return launch(fwd_kernel<D, MODE, KS, VS>, grid, dim3(384), FwdLayout<D, KS, VS>::SMEM_ALLOC, st,
+                  mq, mk, mv, p);
 }
 
 enum BwdParts : int { kPartDq = 1, kPartDkdv = 2 };
@@ -143,14 +144,15 @@ sigattn_status bwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
                         const CUtensorMap &mdo, const BwdParams &p, int Z, int L, int H,
                         int parts, cudaStream_t st) {
     dim3 grid((L + 127) / 128, H, Z);
-    constexpr size_t smem = BwdLayout<D, kBwdStages>::SMEM_ALLOC;
+    constexpr int SX = BwdStages<D>::X, SY = BwdStages<D>::Y;
+    constexpr size_t smem = BwdLayout<D, SX, SY>::SMEM_ALLOC;
     if (parts & kPartDq) {
-        sigattn_status s = launch(bwd_dq_kernel<D, MODE, kBwdStages>, grid, dim3(384), smem, st, mq,
+        sigattn_status s = launch(bwd_dq_kernel<D, MODE, SX, SY>, grid, dim3(384), smem, st, mq,
                                   mk, mv, mdo, p);
         if (s != SIGATTN_OK) return s;
     }
     if (parts & kPartDkdv)
-        return launch(bwd_dkdv_kernel<D, MODE, kBwdStages>, grid, dim3(384), smem, st, mq, mk, mv,
+        return launch(bwd_dkdv_kernel<D, MODE, SX, SY>, grid, dim3(384), smem, st, mq, mk, mv,
                       mdo, p);
     return SIGATTN_OK;
 }
@@ -360,5 +362,20 @@ const char *sigattn_last_cuda_error(void) {
 }
 
 int sigattn_version(void) { return 100; }
+
+#ifdef SIGATTN_TRACE
+// Diagnostic build only: copies the timeline trace (see sm100.cuh) to host
+// memory `dst` of `n` uint64 entries and clears it on the device.
+int sigattn_trace_dump(unsigned long long *dst, int n) {
+    const int total = kTraceRoles * kTraceSteps * kTraceEvents;
+    if (dst == nullptr || n < total) return -1;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -2;
+    if (cudaMemcpyFromSymbol(dst, g_sigattn_trace, sizeof(unsigned long long) * total) != cudaSuccess)
+        return -3;
+    static unsigned long long zeros[kTraceRoles * kTraceSteps * kTraceEvents];
+    if (cudaMemcpyToSymbol(g_sigattn_trace, zeros, sizeof zeros) != cudaSuccess) return -4;
+    return total;
+}
+#endif
 
 }  // extern "C"

@@ -55,7 +55,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 // suspended by the hardware for up to `kSuspendHintNs` (it wakes as soon as the
 // phase completes), so waiting roles do not take issue slots from the warps
 // that share their scheduler.
-constexpr uint32_t kSuspendHintNs = 20000;
+#ifndef SIGATTN_SUSPEND_HINT_NS
+#define SIGATTN_SUSPEND_HINT_NS 20000
+#endif
+constexpr uint32_t kSuspendHintNs = SIGATTN_SUSPEND_HINT_NS;
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
@@ -321,4 +324,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rh(float lo, float hi) {
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
+}  // namespace sigattn
+
+// ---------------------------------------------------------------- timeline trace
+// Built only with -DSIGATTN_TRACE (libsigattn_trace.so, a diagnostic build): one
+// CTA per launch (the one at blockIdx (gridDim.x / 2, 0, 0)) records clock64()
+// at each role's waits and hand-offs into g_sigattn_trace[role][step][event],
+// read back with sigattn_trace_dump().  The default build compiles it away.
+namespace sigattn {
+constexpr int kTraceRoles = 4, kTraceSteps = 256, kTraceEvents = 8;
+#ifdef SIGATTN_TRACE
+__device__ unsigned long long g_sigattn_trace[kTraceRoles * kTraceSteps * kTraceEvents];
+__device__ __forceinline__ bool trace_cta() {
+    return blockIdx.x == gridDim.x / 2 && blockIdx.y == 0 && blockIdx.z == 0;
+}
+__device__ __forceinline__ void trace(int role, int step, int ev) {
+    if (trace_cta() && (threadIdx.x & 31) == 0 && step < kTraceSteps)
+        g_sigattn_trace[(role * kTraceSteps + step) * kTraceEvents + ev] = clock64();
+}
+#else
+__device__ __forceinline__ void trace(int, int, int) {}
+#endif
 }  // namespace sigattn
