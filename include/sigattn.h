@@ -59,7 +59,8 @@ typedef enum {
     SIGATTN_ERR_MISALIGNED = 5,           /* a base pointer is not 16-byte aligned */
     SIGATTN_ERR_CUDA = 6,                 /* a CUDA runtime/driver call failed */
     SIGATTN_ERR_TIMEOUT = 7,              /* device: a bounded wait ran out */
-    SIGATTN_ERR_SEQLEN_RANGE = 8          /* device: a length was outside [0, L] */
+    SIGATTN_ERR_SEQLEN_RANGE = 8,         /* device: a length was outside [0, L] */
+    SIGATTN_ERR_TOO_LARGE = 9             /* a size exceeds a fixed limit (sigattn_fwd_noalloc) */
 } sigattn_status;
 
 typedef enum {
@@ -144,6 +145,41 @@ sigattn_status sigattn_set_wait_timeout_ns(uint64_t ns);
  * SIGATTN_ERR_TIMEOUT recorded in the status word and leave the context
  * usable.  Exercises the failure path of the bounded waits. */
 sigattn_status sigattn_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
+
+/* Forward for callers that must not allocate device memory.
+ *
+ * No counterpart in the paper; this is a deployment convenience.  Some
+ * callers cannot call cudaMalloc at the time they run attention: code
+ * running inside a CUDA-graph capture, inside a framework whose caching
+ * allocator owns all device memory, or in a service that reserves its memory
+ * at start-up and forbids allocation on the request path.  Such callers
+ * often also have the per-sample lengths only on the host.  This entry point
+ * computes exactly what sigattn_fwd computes, with the same kernel, but takes
+ * seqlens_q / seqlens_k as HOST int32[Z] arrays and never allocates: the
+ * lengths and the kernel's device status word live in a fixed array in the
+ * library's own device memory (a file-scope __device__ array, loaded with
+ * the module, present on every GPU that loads the library until exit).
+ *
+ * Limits and behaviour:
+ *  - Z <= SIGATTN_NOALLOC_MAX_Z (8192), else SIGATTN_ERR_TOO_LARGE and
+ *    nothing is launched.  Lengths are checked on the host: any value
+ *    outside [0, L] returns SIGATTN_ERR_SEQLEN_RANGE before any launch.
+ *  - The host arrays may be reused as soon as the call returns (they are
+ *    staged with cudaMemcpyAsync from pageable memory).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call shares the one array, and it keeps the last call's contents
+ *    (the status word is cleared at the start of each call): calls whose
+ *    work overlaps on the GPU (different streams, or devices driven from
+ *    several threads at once) race on it and must be serialised by the
+ *    caller.  A wait that runs out inside the kernel is recorded in that
+ *    array's status word only; sigattn_last_device_status does not see it.
+ * Other arguments, layout and errors as sigattn_fwd. */
+#define SIGATTN_NOALLOC_MAX_Z 8192
+sigattn_status sigattn_fwd_noalloc(const void *q, const void *k, const void *v, void *o,
+                                   const int32_t *host_seqlens_q, const int32_t *host_seqlens_k,
+                                   int Z, int L, int H, int D, float alpha, float bias,
+                                   sigattn_dtype dtype, void *stream);
 
 /* Text of the CUDA error behind the most recent SIGATTN_ERR_CUDA returned
  * by any call in this process (static string; "no error" if none). */

@@ -21,7 +21,7 @@ __all__ = [
     "SigattnError", "fwd", "bwd", "sigmoid_eval", "set_sigmoid_mode", "get_sigmoid_mode",
     "last_device_status", "set_wait_timeout_ns", "selftest_wait_timeout", "status_string",
     "version", "library_path", "load_library", "SIGMOID_TANH", "SIGMOID_EXP", "EXPORTS",
-    "SigmoidAttention", "bwd_dq", "bwd_dkdv", "last_cuda_error",
+    "SigmoidAttention", "bwd_dq", "bwd_dkdv", "last_cuda_error", "fwd_noalloc", "NOALLOC_MAX_Z",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,8 +37,10 @@ STATUS_NAMES = {
     0: "SIGATTN_OK", 1: "SIGATTN_ERR_INVALID_ARG", 2: "SIGATTN_ERR_UNSUPPORTED_HEADDIM",
     3: "SIGATTN_ERR_UNSUPPORTED_DTYPE", 4: "SIGATTN_ERR_UNSUPPORTED_DEVICE",
     5: "SIGATTN_ERR_MISALIGNED", 6: "SIGATTN_ERR_CUDA", 7: "SIGATTN_ERR_TIMEOUT",
-    8: "SIGATTN_ERR_SEQLEN_RANGE",
+    8: "SIGATTN_ERR_SEQLEN_RANGE", 9: "SIGATTN_ERR_TOO_LARGE",
 }
+
+NOALLOC_MAX_Z = 8192   # SIGATTN_NOALLOC_MAX_Z
 
 # every symbol include/sigattn.h declares
 EXPORTS = (
@@ -46,6 +48,7 @@ EXPORTS = (
     "sigattn_set_sigmoid_mode", "sigattn_get_sigmoid_mode", "sigattn_sigmoid_eval",
     "sigattn_last_device_status", "sigattn_set_wait_timeout_ns", "sigattn_selftest_wait_timeout",
     "sigattn_last_cuda_error", "sigattn_status_string", "sigattn_version",
+    "sigattn_fwd_noalloc",
 )
 
 
@@ -83,6 +86,8 @@ def load_library():
                                          ci, vp]
         lib.sigattn_bwd_dkdv.restype = ci
         lib.sigattn_last_cuda_error.restype = ctypes.c_char_p
+        lib.sigattn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf, ci, vp]
+        lib.sigattn_fwd_noalloc.restype = ci
         lib.sigattn_set_sigmoid_mode.argtypes = [ci]
         lib.sigattn_set_sigmoid_mode.restype = ci
         lib.sigattn_get_sigmoid_mode.restype = ci
@@ -200,6 +205,33 @@ def bwd_dkdv(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, dk=
         seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, L, H, D, float(alpha), float(bias),
         _dtype_code(q), _stream_ptr(q)), "sigattn_bwd_dkdv")
     return dk, dv
+
+
+def fwd_noalloc(q, k, v, seqlens_q, seqlens_k, alpha: float, bias: float, out=None):
+    """Forward for callers that cannot allocate device memory: the same result as
+    ``fwd``, with the lengths given on the host (numpy int32 arrays or CPU
+    tensors) and staged in the library's fixed device array instead of any
+    allocation (see sigattn_fwd_noalloc in include/sigattn.h).  ``out`` should be
+    preallocated by such callers; Z is limited to NOALLOC_MAX_Z."""
+    import numpy as np
+    import torch
+    _check_inputs([q, k, v], [])
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_inputs([q, out], [])
+    nq = np.ascontiguousarray(np.asarray(seqlens_q.cpu() if hasattr(seqlens_q, "cpu") else seqlens_q,
+                                         dtype=np.int32).reshape(-1))
+    nk = np.ascontiguousarray(np.asarray(seqlens_k.cpu() if hasattr(seqlens_k, "cpu") else seqlens_k,
+                                         dtype=np.int32).reshape(-1))
+    Z, L, H, D = (int(s) for s in q.shape)
+    if nq.shape[0] != Z or nk.shape[0] != Z:
+        raise ValueError("seqlens must have Z entries")
+    _check(load_library().sigattn_fwd_noalloc(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+        nq.ctypes.data_as(ctypes.c_void_p), nk.ctypes.data_as(ctypes.c_void_p), Z, L, H, D,
+        float(alpha), float(bias), _dtype_code(q), _stream_ptr(q)), "sigattn_fwd_noalloc")
+    return out
 
 
 def last_cuda_error() -> str:

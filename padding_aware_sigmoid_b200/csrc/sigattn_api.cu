@@ -346,6 +346,7 @@ const char *sigattn_status_string(sigattn_status s) {
         case SIGATTN_ERR_CUDA: return "SIGATTN_ERR_CUDA";
         case SIGATTN_ERR_TIMEOUT: return "SIGATTN_ERR_TIMEOUT";
         case SIGATTN_ERR_SEQLEN_RANGE: return "SIGATTN_ERR_SEQLEN_RANGE";
+        case SIGATTN_ERR_TOO_LARGE: return "SIGATTN_ERR_TOO_LARGE";
     }
     return "SIGATTN_UNKNOWN_STATUS";
 }
@@ -362,6 +363,101 @@ const char *sigattn_last_cuda_error(void) {
 }
 
 int sigattn_version(void) { return 100; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Scratch-free forward (sigattn_fwd_noalloc): the lengths and the status word
+// of its kernel live in this fixed device array instead of caller or library
+// allocations.  Layout (int32): [0] status word, [64, 64 + Z) n_q,
+// [64 + MAX_Z, 64 + MAX_Z + Z) n_k.
+namespace {
+constexpr int kNoallocHeader = 64;   // 256 bytes: status word and padding
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocHeader + 2 * SIGATTN_NOALLOC_MAX_Z];
+
+std::mutex g_noalloc_mu;
+int32_t *g_noalloc_ptr[kMaxDevices] = {};   // device address of the array, per device
+
+// Looks up (once per device, with that device current) where the array lives
+// on the device; the host-side name is only a stand-in for it.
+sigattn_status noalloc_scratch(int dev, int32_t **ptr) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) return cuda_fail(e);
+        g_noalloc_ptr[dev] = static_cast<int32_t *>(p);
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return SIGATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+sigattn_status sigattn_fwd_noalloc(const void *q, const void *k, const void *v, void *o,
+                                   const int32_t *host_seqlens_q, const int32_t *host_seqlens_k,
+                                   int Z, int L, int H, int D, float alpha, float bias,
+                                   sigattn_dtype dtype, void *stream) {
+    bool empty = false;
+    sigattn_status s = check_shape(Z, L, H, D, dtype, &empty);
+    if (s != SIGATTN_OK) return s;
+    if (Z > SIGATTN_NOALLOC_MAX_Z) return SIGATTN_ERR_TOO_LARGE;
+    if (empty) return SIGATTN_OK;
+    if (!q || !k || !v || !o || !host_seqlens_q || !host_seqlens_k) return SIGATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return SIGATTN_ERR_MISALIGNED;
+    for (int z = 0; z < Z; ++z)
+        if (host_seqlens_q[z] < 0 || host_seqlens_q[z] > L || host_seqlens_k[z] < 0 ||
+            host_seqlens_k[z] > L)
+            return SIGATTN_ERR_SEQLEN_RANGE;
+    // device and capability without the status-buffer allocation of device_state()
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(e);
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+        return cuda_fail(e);
+    if (dtype == SIGATTN_BF16 && major * 10 + minor != 100) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
+    int32_t *scratch = nullptr;
+    if ((s = noalloc_scratch(dev, &scratch)) != SIGATTN_OK) return s;
+    int32_t *status = scratch;
+    int32_t *nq = scratch + kNoallocHeader;
+    int32_t *nk = scratch + kNoallocHeader + SIGATTN_NOALLOC_MAX_Z;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the array keeps the previous call's contents: clear the status word
+    if ((e = cudaMemsetAsync(status, 0, sizeof(int32_t), st)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemcpyAsync(nq, host_seqlens_q, sizeof(int32_t) * Z, cudaMemcpyHostToDevice, st)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(nk, host_seqlens_k, sizeof(int32_t) * Z, cudaMemcpyHostToDevice, st)) !=
+            cudaSuccess)
+        return cuda_fail(e);
+    if (dtype == SIGATTN_FP32) {
+        F32Params p{static_cast<const float *>(q), static_cast<const float *>(k),
+                    static_cast<const float *>(v), nullptr, static_cast<float *>(o), nullptr,
+                    nullptr, nullptr, nq, nk, Z, L, H, alpha, bias, status};
+        const int64_t rows = static_cast<int64_t>(Z) * L * H;
+        dim3 grid(static_cast<unsigned>((rows + 7) / 8));
+        return D == 64 ? launch(f32_fwd_kernel<64>, grid, dim3(256), 0, st, p)
+                       : launch(f32_fwd_kernel<128>, grid, dim3(256), 0, st, p);
+    }
+    if ((s = get_encoder()) != SIGATTN_OK) return s;
+    CUtensorMap mq, mk, mv;
+    if ((s = encode_bf16_map(&mq, q, Z, L, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
+    FwdParams p{static_cast<__nv_bfloat16 *>(o), nq, nk, L, H, alpha, bias, status,
+                g_timeout_ns.load()};
+    const int mode = g_sigmoid_mode.load();
+    if (D == 128)
+        return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
+                                    : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
+    return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
+                                : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
+}
 
 #ifdef SIGATTN_TRACE
 // Diagnostic build only: copies the timeline trace (see sm100.cuh) to host
