@@ -139,9 +139,9 @@ __device__ __forceinline__ void mask_packed(uint32_t (&pk)[32], int col0, int va
 // Per key tile j the warpgroups (1) read S_j and release it, keeping
 // sigma'(S_j) in registers, then (2) read dP_j and write dS_j = sigma' dP_j
 // over dP_j.  The MMA thread issues S_{j+1} as soon as S_j is released and
-// dP_{j+1} into the other dP buffer (free once dQ += dS_{j-1} K_{j-1} has
-// finished), then dQ += dS_j K_j when dS_j is ready: neither warpgroup phase
-// waits on the MMA that consumes the previous tile.  The two warpgroups take
+// dP_{j+1} into the other dP buffer (its dS_{j-1} is read by an earlier MMA of
+// the same thread, and MMAs run in issue order), then dQ += dS_j K_j when dS_j
+// is ready: neither warpgroup phase waits on the MMA of the previous tile.  The two warpgroups take
 // turns for the sigma' phase (warpgroup 0 first), so that it has the MUFU to
 // itself while the other warpgroup forms dS.
 // ============================================================================
@@ -283,8 +283,8 @@ __global__ void __launch_bounds__(384, 1)
                     issue_xyT(kColS, sQ, kslot(j + 1));
                     mma_commit(s_full);
                     if (!(ok = mbar_wait(&y_full[(j + 1) % SY], ((j + 1) / SY) & 1, wctx))) break;
-                    // buffer (j+1) % 2 holds dS_{j-1} until dQ += dS_{j-1} K_{j-1} is done
-                    if (j > 0 && !(ok = mbar_wait(dq_done, (j - 1) & 1, wctx))) break;
+                    // buffer (j+1) % 2 still holds dS_{j-1}: dQ += dS_{j-1} K_{j-1} was
+                    // issued earlier by this thread and MMAs run in issue order
                     trace(1, j, 1);
                     tc_fence_after();
                     issue_xyT((j + 1) & 1 ? kColDP1 : kColDP0, sDO, vslot(j + 1));
@@ -301,7 +301,6 @@ __global__ void __launch_bounds__(384, 1)
                     mma_ts(tmem + kColDQ, tmem + dcol + packed_col(kk),
                            smem_desc_sw128(sK + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_q,
                            (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(dq_done);
                 mma_commit(&x_empty[j % SX]);             // K_j: S_j and dQ_j done
             }
             mma_commit(drain);
@@ -366,7 +365,8 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive(&ds_ready[j & 1]);
                 if (quarter == 0) trace(2 + w, j, 6);
             }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dq_done, (nkv - 1) & 1, wctx));
+            // every MMA of this CTA has finished once the MMA thread's final commit lands
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
             if (ok) {
                 tc_fence_after();
                 store_row_from_tmem<D>(tmem + lane_bits + kColDQ, drow, row < L, row < nq,
@@ -393,9 +393,9 @@ __global__ void __launch_bounds__(384, 1)
 // TMEM: [0,128) S^T / P^T, [128,256) dP^T / dS^T, [256,256+D) dV, [256+D,256+2D) dK.
 //
 // The warpgroups publish P^T first (it needs S^T only) and dS^T second; the
-// MMA order per query tile is dV_i, S^T_{i+1} (after dV_i consumed P^T_i),
-// dK_i, dP^T_{i+1} (after dK_i consumed dS^T_i), so the sigma work on i+1
-// overlaps dK_i.
+// MMA order per query tile is dV_i, S^T_{i+1} (over P^T_i, which dV_i has read:
+// MMAs from one thread run in issue order), dK_i, dP^T_{i+1} (over dS^T_i), so
+// the sigma work on i+1 overlaps dK_i.
 // ============================================================================
 template <int D, int MODE, int SX, int SY>
 __global__ void __launch_bounds__(384, 1)
@@ -484,10 +484,12 @@ __global__ void __launch_bounds__(384, 1)
                                              i, h, z, wctx))
                     break;
                 ix = i + 1;
+                trace(0, i, 0);
                 if (!ring_load<SY, Lay::NSUB>(&tmDO, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
                                              i, h, z, wctx))
                     break;
                 iy = i + 1;
+                trace(0, i, 1);
             }
             mbar_wait_drain(res_full, 0, p.timeout_ns);
             ring_drain<SX>(x_full, ix, p.timeout_ns);
@@ -529,25 +531,28 @@ __global__ void __launch_bounds__(384, 1)
             for (int i = 0; ok && i < nqt; ++i) {
                 const bool more = i + 1 < nqt;
                 if (!(ok = mbar_wait(p_ready, i & 1, wctx))) break;
+                trace(1, i, 0);
                 tc_fence_after();
                 issue_acc(Lay::COL_ACC0, Lay::COL_S, doslot(i), i == 0);      // dV += P^T dO_i
-                mma_commit(dv_done);
                 mma_commit(&y_empty[i % SY]);                                 // dO_i: dP^T_i, dV_i done
                 if (more) {
+                    // S^T_{i+1} overwrites P^T_i, read by the dV MMA just issued
+                    // (MMAs run in issue order)
                     if (!(ok = mbar_wait(&x_full[(i + 1) % SX], ((i + 1) / SX) & 1, wctx))) break;
-                    if (!(ok = mbar_wait(dv_done, i & 1, wctx))) break;   // P^T_i consumed
+                    trace(1, i, 1);
                     tc_fence_after();
                     issue_xyT(Lay::COL_S, sK, qslot(i + 1));
                     mma_commit(s_full);
                 }
                 if (!(ok = mbar_wait(ds_ready, i & 1, wctx))) break;
+                trace(1, i, 2);
                 tc_fence_after();
                 issue_acc(Lay::COL_ACC1, Lay::COL_DP, qslot(i), i == 0);      // dK += dS^T Q_i
-                mma_commit(dk_done);
                 mma_commit(&x_empty[i % SX]);                                 // Q_i: S^T_i, dK_i done
                 if (more) {
+                    // dP^T_{i+1} overwrites dS^T_i, read by the dK MMA just issued
                     if (!(ok = mbar_wait(&y_full[(i + 1) % SY], ((i + 1) / SY) & 1, wctx))) break;
-                    if (!(ok = mbar_wait(dk_done, i & 1, wctx))) break;   // dS^T_i consumed
+                    trace(1, i, 3);
                     tc_fence_after();
                     issue_xyT(Lay::COL_DP, sV, doslot(i + 1));
                     mma_commit(dp_full);
@@ -571,8 +576,10 @@ __global__ void __launch_bounds__(384, 1)
                 const int qvalid = nq - i * 128;
                 float2 g[32];
                 {
+                    if (quarter == 0) trace(2 + w, i, 0);
                     ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
                     if (!ok) break;
+                    if (quarter == 0) trace(2 + w, i, 1);
                     tc_fence_after();
                     uint32_t r[64];
                     tmem_ld64(tmem + lane_bits + Lay::COL_S + 64 * w, r);
@@ -589,9 +596,11 @@ __global__ void __launch_bounds__(384, 1)
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(p_ready);
+                    if (quarter == 0) trace(2 + w, i, 2);
                 }
                 ok = __all_sync(0xffffffffu, mbar_wait(dp_full, i & 1, wctx));
                 if (!ok) break;
+                if (quarter == 0) trace(2 + w, i, 3);
                 tc_fence_after();
                 uint32_t d[64];
                 tmem_ld64(tmem + lane_bits + Lay::COL_DP + 64 * w, d);
@@ -606,10 +615,10 @@ __global__ void __launch_bounds__(384, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ds_ready);
+                if (quarter == 0) trace(2 + w, i, 4);
             }
-            if (ok)
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(w == 0 ? dv_done : dk_done, (nqt - 1) & 1, wctx));
+            // every MMA of this CTA has finished once the MMA thread's final commit lands
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
             if (ok) {
                 tc_fence_after();
                 store_row_from_tmem<D>(tmem + lane_bits + (w == 0 ? Lay::COL_ACC0 : Lay::COL_ACC1), dst,

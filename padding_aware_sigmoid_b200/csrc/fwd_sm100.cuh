@@ -20,12 +20,18 @@
 //
 // Per key tile j the MMA thread issues S0 = Q0 K_j^T, S1 = Q1 K_j^T, then
 // O0 += P0 V_j, O1 += P1 V_j as the warpgroups publish P.  S_t of tile j+1 is
-// issued only after O_t += P_t V_j has completed (P_t aliases S_t); the other
-// query tile's work fills the tensor pipe meanwhile.
+// issued right after O_t += P_t V_j (P_t aliases S_t; MMAs from one thread run
+// in issue order); the other query tile's work fills the tensor pipe meanwhile.
 #pragma once
 
 #include "sm100.cuh"
 #include "sigmoid.cuh"
+
+// Which half of a tile's sigma work (0 or 1) hands the MUFU token to the other
+// warpgroup once its last MUFU op is issued.
+#ifndef SIGATTN_FWD_TOKEN_HALF
+#define SIGATTN_FWD_TOKEN_HALF 1
+#endif
 
 namespace sigattn {
 
@@ -174,12 +180,14 @@ __global__ void __launch_bounds__(384, 1)
                     tma_load_4d(&tmK, &k_full[sk], sK + sk * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
                                 64 * s, h, j * Lay::BN, z);
                 issued_k = j + 1;
+                trace(0, j, 0);
                 if (j >= VS && !mbar_wait(&v_empty[sv], ((j / VS) - 1) & 1, wctx)) break;
                 mbar_arrive_expect_tx(&v_full[sv], Lay::TILE_BYTES);
                 for (int s = 0; s < Lay::NSUB; ++s)
                     tma_load_4d(&tmV, &v_full[sv], sV + sv * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
                                 64 * s, h, j * Lay::BN, z);
                 issued_v = j + 1;
+                trace(0, j, 1);
             }
             // Every issued load must land before the CTA's shared memory is released.
             mbar_wait_drain(q_full, 0, p.timeout_ns);
@@ -217,12 +225,13 @@ __global__ void __launch_bounds__(384, 1)
                     mma_ts(d_tmem, a_tmem + kk * 8,
                            smem_desc_sw128(vbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_o,
                            (!first || kk > 0) ? 1u : 0u);
-                mma_commit(&pv_done[t]);
             };
             // Order per key tile j: PV0_j, S0_{j+1}, PV1_j, S1_{j+1}.  Tile 0's next
             // scores never wait for tile 1's P, so the two sigma warpgroups can
             // alternate while the tensor pipe works on the other tile.  S_t of
-            // j+1 overwrites P_t of j, so it is issued only after PV_t_j completed.
+            // j+1 overwrites P_t of j right after O_t += P_t V_j is issued: MMAs
+            // issued by one thread execute in issue order, so the P.V MMA has read
+            // P_t before the next scores are written over it.
             bool ok = mbar_wait(q_full, 0, wctx) && mbar_wait(&k_full[0], 0, wctx);
             if (ok) {
                 tc_fence_after();
@@ -236,14 +245,16 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t vbase = sV + stv * Lay::TILE_BYTES;
                 const uint32_t knext = sK + stk * Lay::TILE_BYTES;
                 if (!(ok = mbar_wait(&v_full[stv], (j / VS) & 1, wctx))) break;
+                trace(1, j, 0);
                 for (int t = 0; t < ntiles; ++t) {
                     if (!(ok = mbar_wait(&p_full[t], j & 1, wctx))) break;
+                    trace(1, j, 1 + 2 * t);
                     tc_fence_after();
                     issue_pv(t, vbase, j == 0);
                     if (t == ntiles - 1) mma_commit(&v_empty[stv]);
                     if (more) {
                         if (t == 0 && !(ok = mbar_wait(&k_full[stk], ((j + 1) / KS) & 1, wctx))) break;
-                        if (!(ok = mbar_wait(&pv_done[t], j & 1, wctx))) break;
+                        trace(1, j, 2 + 2 * t);
                         tc_fence_after();
                         issue_s(t, knext);
                         if (t == ntiles - 1) mma_commit(&k_empty[stk]);
@@ -274,13 +285,16 @@ __global__ void __launch_bounds__(384, 1)
                 // The two warpgroups take turns (tile 0 first) so that each sigma
                 // phase has the MUFU to itself while the tensor pipe runs the other
                 // tile's P.V and next scores.
+                if (quarter == 0) trace(2 + t, j, 0);
+                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wctx));
+                if (!ok) break;
+                if (quarter == 0) trace(2 + t, j, 1);
                 if (pingpong && (t == 1 || j > 0)) {
                     ok = __all_sync(0xffffffffu,
                                     mbar_wait(&turn[t], (t == 0 ? j - 1 : j) & 1, wctx));
                     if (!ok) break;
                 }
-                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wctx));
-                if (!ok) break;
+                if (quarter == 0) trace(2 + t, j, 2);
                 tc_fence_after();
                 const int kvalid = nk - j * Lay::BN;   // keys of this tile below n_k
 #pragma unroll
@@ -294,12 +308,11 @@ __global__ void __launch_bounds__(384, 1)
                     for (int i = 0; i < 32; ++i) {
                         const float2 pr = sigma2<MODE>(
                             scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
-#ifdef SIGATTN_FWD_PACK_CVT
                         pk[i] = pack_bf16x2(pr.x, pr.y);
-#else
-                        pk[i] = pack_bf16x2_rh(pr.x, pr.y);
-#endif
                     }
+                    // the last MUFU op of this tile is issued: hand the MUFU to the
+                    // other warpgroup before packing and storing
+                    if (half == SIGATTN_FWD_TOKEN_HALF && pingpong) mbar_arrive(&turn[t ^ 1]);
                     if (kvalid < Lay::BN) {
                         // last tile: keys at or beyond n_k weigh exactly zero
 #pragma unroll
@@ -313,12 +326,14 @@ __global__ void __launch_bounds__(384, 1)
                     // P columns [32 half, 32 half + 32) lie over S columns already read
                     tmem_st32(tS + 32 * half, pk);
                 }
+                if (quarter == 0) trace(2 + t, j, 3);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[t]);
-                if (pingpong) mbar_arrive(&turn[t ^ 1]);
+                if (quarter == 0) trace(2 + t, j, 4);
             }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[t], (nkv - 1) & 1, wctx));
+            // every MMA of this CTA has finished once the MMA thread's final commit lands
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
             if (ok) {
                 tc_fence_after();
                 const bool valid = row < nq;

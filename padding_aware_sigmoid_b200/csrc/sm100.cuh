@@ -311,16 +311,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Two finite floats to packed bf16 (lo in the low half),
-// rounding half away from zero: add half an ulp of bf16 to the bit pattern and
-// keep the high halves.  Differs from round-to-nearest-even only on exact
-// ties, and runs on the integer pipe instead of the conversion unit.
-__device__ __forceinline__ uint32_t pack_bf16x2_rh(float lo, float hi) {
-    const uint32_t a = __float_as_uint(lo) + 0x8000u;
-    const uint32_t b = __float_as_uint(hi) + 0x8000u;
-    return __byte_perm(a, b, 0x7632);
-}
-
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
