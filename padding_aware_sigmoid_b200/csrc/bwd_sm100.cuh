@@ -5,8 +5,8 @@
 //   dP = dO V^T,  dS = sigma'(S) dP  (sigma' = P (1 - P)),
 //   dQ = alpha dS K,   dK = alpha dS^T Q,   dV = P^T dO.
 //
-// Both kernels share the forward's structure: warp 0 issues TMA loads, one
-// thread of warp 1 issues tcgen05.mma, and two warpgroups (warps 4-7 and
+// Both kernels share the forward's structure: warps 0 and 2 issue TMA loads
+// (one ring each), one thread of warp 1 issues tcgen05.mma, and two warpgroups (warps 4-7 and
 // 8-11) turn the fp32 score tiles in TMEM into bf16 operands, each owning 64
 // of the 128 columns (thread = TMEM lane = tile row).  The bf16 results are
 // written back into TMEM over columns their own warpgroup has already read,
@@ -231,19 +231,26 @@ __global__ void __launch_bounds__(384, 1)
                 tma_load_4d(&tmQ, res_full, sQ + s * Lay::SUB_BYTES, 64 * s, h, qtile * 128, z);
                 tma_load_4d(&tmDO, res_full, sDO + s * Lay::SUB_BYTES, 64 * s, h, qtile * 128, z);
             }
-            int ix = 0, iy = 0;
+            int ix = 0;
             for (int j = 0; j < nkv; ++j) {
                 if (!ring_load<SX, Lay::NSUB>(&tmK, x_full, x_empty, smem + Lay::OFF_X, Lay::TILE_BYTES,
                                              j, h, z, wctx))
                     break;
                 ix = j + 1;
+            }
+            mbar_wait_drain(res_full, 0, p.timeout_ns);
+            ring_drain<SX>(x_full, ix, p.timeout_ns);
+        }
+    } else if (warp == 2) {
+        // V_j ring, fed by its own thread so it never waits behind a key slot
+        if (work && lane == 0) {
+            int iy = 0;
+            for (int j = 0; j < nkv; ++j) {
                 if (!ring_load<SY, Lay::NSUB>(&tmV, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
                                              j, h, z, wctx))
                     break;
                 iy = j + 1;
             }
-            mbar_wait_drain(res_full, 0, p.timeout_ns);
-            ring_drain<SX>(x_full, ix, p.timeout_ns);
             ring_drain<SY>(y_full, iy, p.timeout_ns);
         }
     } else if (warp == 1) {
@@ -478,21 +485,28 @@ __global__ void __launch_bounds__(384, 1)
                 tma_load_4d(&tmK, res_full, sK + s * Lay::SUB_BYTES, 64 * s, h, ktile * 128, z);
                 tma_load_4d(&tmV, res_full, sV + s * Lay::SUB_BYTES, 64 * s, h, ktile * 128, z);
             }
-            int ix = 0, iy = 0;
+            int ix = 0;
             for (int i = 0; i < nqt; ++i) {
                 if (!ring_load<SX, Lay::NSUB>(&tmQ, x_full, x_empty, smem + Lay::OFF_X, Lay::TILE_BYTES,
                                              i, h, z, wctx))
                     break;
                 ix = i + 1;
                 trace(0, i, 0);
+            }
+            mbar_wait_drain(res_full, 0, p.timeout_ns);
+            ring_drain<SX>(x_full, ix, p.timeout_ns);
+        }
+    } else if (warp == 2) {
+        // dO_i ring, fed by its own thread so it never waits behind a query slot
+        if (work && lane == 0) {
+            int iy = 0;
+            for (int i = 0; i < nqt; ++i) {
                 if (!ring_load<SY, Lay::NSUB>(&tmDO, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
                                              i, h, z, wctx))
                     break;
                 iy = i + 1;
                 trace(0, i, 1);
             }
-            mbar_wait_drain(res_full, 0, p.timeout_ns);
-            ring_drain<SX>(x_full, ix, p.timeout_ns);
             ring_drain<SY>(y_full, iy, p.timeout_ns);
         }
     } else if (warp == 1) {

@@ -9,7 +9,8 @@
 // section 4).
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles once, then K_j / V_j into a ring of stages
+//   warp 0      TMA producer: Q tiles once, then K_j into the key ring
+//   warp 2      TMA producer: V_j into the value ring
 //   warp 1      owns TMEM; one thread issues every tcgen05.mma
 //   warps 4-7   sigma warpgroup of query tile 0 (thread = query row)
 //   warps 8-11  sigma warpgroup of query tile 1
@@ -171,9 +172,9 @@ __global__ void __launch_bounds__(384, 1)
                 for (int s = 0; s < Lay::NSUB; ++s)
                     tma_load_4d(&tmQ, q_full, sQ + t * Lay::TILE_BYTES + s * Lay::SUB_BYTES,
                                 64 * s, h, (qtile0 + t) * Lay::BM, z);
-            int issued_k = 0, issued_v = 0;
+            int issued_k = 0;
             for (int j = 0; j < nkv; ++j) {
-                const int sk = j % KS, sv = j % VS;
+                const int sk = j % KS;
                 if (j >= KS && !mbar_wait(&k_empty[sk], ((j / KS) - 1) & 1, wctx)) break;
                 mbar_arrive_expect_tx(&k_full[sk], Lay::TILE_BYTES);
                 for (int s = 0; s < Lay::NSUB; ++s)
@@ -181,6 +182,21 @@ __global__ void __launch_bounds__(384, 1)
                                 64 * s, h, j * Lay::BN, z);
                 issued_k = j + 1;
                 trace(0, j, 0);
+            }
+            // Every issued load must land before the CTA's shared memory is released.
+            mbar_wait_drain(q_full, 0, p.timeout_ns);
+            for (int j = (issued_k > KS ? issued_k - KS : 0); j < issued_k; ++j)
+                mbar_wait_drain(&k_full[j % KS], (j / KS) & 1, p.timeout_ns);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ value producer
+        // V_j is released later than K_j, so its ring is fed by its own thread
+        // and never waits behind a key slot.
+        if (work && lane == 0) {
+            uint8_t *sV = smem + Lay::OFF_V;
+            int issued_v = 0;
+            for (int j = 0; j < nkv; ++j) {
+                const int sv = j % VS;
                 if (j >= VS && !mbar_wait(&v_empty[sv], ((j / VS) - 1) & 1, wctx)) break;
                 mbar_arrive_expect_tx(&v_full[sv], Lay::TILE_BYTES);
                 for (int s = 0; s < Lay::NSUB; ++s)
@@ -189,10 +205,6 @@ __global__ void __launch_bounds__(384, 1)
                 issued_v = j + 1;
                 trace(0, j, 1);
             }
-            // Every issued load must land before the CTA's shared memory is released.
-            mbar_wait_drain(q_full, 0, p.timeout_ns);
-            for (int j = (issued_k > KS ? issued_k - KS : 0); j < issued_k; ++j)
-                mbar_wait_drain(&k_full[j % KS], (j / KS) & 1, p.timeout_ns);
             for (int j = (issued_v > VS ? issued_v - VS : 0); j < issued_v; ++j)
                 mbar_wait_drain(&v_full[j % VS], (j / VS) & 1, p.timeout_ns);
         }
