@@ -141,9 +141,9 @@ __device__ __forceinline__ void mask_packed(uint32_t (&pk)[32], int col0, int va
 // over dP_j.  The MMA thread issues S_{j+1} as soon as S_j is released and
 // dP_{j+1} into the other dP buffer (its dS_{j-1} is read by an earlier MMA of
 // the same thread, and MMAs run in issue order), then dQ += dS_j K_j when dS_j
-// is ready: neither warpgroup phase waits on the MMA of the previous tile.  The two warpgroups take
-// turns for the sigma' phase (warpgroup 0 first), so that it has the MUFU to
-// itself while the other warpgroup forms dS.
+// is ready: neither warpgroup phase waits on the MMA of the previous tile.  Both
+// warpgroups run their sigma' phase at the same time, so that two warps share
+// each SM sub-partition's MUFU (one warp alone leaves it idle between issues).
 // ============================================================================
 template <int D, int MODE, int SX, int SY>
 __global__ void __launch_bounds__(384, 1)
@@ -167,8 +167,7 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t *ds_ready = s_free + 1;          // [2] WGs -> MMA: dS_j in buffer j % 2
     uint64_t *dq_done = ds_ready + 2;         // MMA -> all: dQ += dS_j K_j finished
     uint64_t *drain = dq_done + 1;
-    uint64_t *turn = drain + 1;               // [2] sigma' phase token per warpgroup
-    static_assert(10 <= Lay::MAX_HANDOFF, "barrier count");
+    static_assert(8 <= Lay::MAX_HANDOFF, "barrier count");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -202,8 +201,6 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(&ds_ready[1], 256);
         mbar_init(dq_done, 1);
         mbar_init(drain, 1);
-        mbar_init(&turn[0], 128);
-        mbar_init(&turn[1], 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -336,18 +333,12 @@ __global__ void __launch_bounds__(384, 1)
                     if (quarter == 0) trace(2 + w, j, 2);
                     tc_fence_before();
                     mbar_arrive(s_free);
-                    if (w == 1 || j > 0) {
-                        ok = __all_sync(0xffffffffu,
-                                        mbar_wait(&turn[w], (w == 0 ? j - 1 : j) & 1, wctx));
-                        if (!ok) break;
-                    }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         float2 pr;
                         sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf),
                                           pr, g[i]);
                     }
-                    mbar_arrive(&turn[w ^ 1]);
                 }
                 const uint32_t dcol = (j & 1 ? kColDP1 : kColDP0) + 64 * w;
                 if (quarter == 0) trace(2 + w, j, 3);

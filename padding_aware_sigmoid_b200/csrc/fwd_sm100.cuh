@@ -12,12 +12,15 @@
 //   warp 0      TMA producer: Q tiles once, then K_j into the key ring
 //   warp 2      TMA producer: V_j into the value ring
 //   warp 1      owns TMEM; one thread issues every tcgen05.mma
-//   warps 4-7   sigma warpgroup of query tile 0 (thread = query row)
-//   warps 8-11  sigma warpgroup of query tile 1
+//   warps 4-7   sigma warpgroup 0: keys [0,64) of each tile (thread = query row),
+//               then the epilogue of query tile 0
+//   warps 8-11  sigma warpgroup 1: keys [64,128) of each tile, epilogue of tile 1
 // Tensor memory (512 columns, fp32):
 //   [0,128) S0   [128,256) S1   [256,256+D) O0   [256+D,256+2D) O1
-// P_t (bf16, two per column) overwrites the first 64 columns of S_t and is the
-// TMEM-resident A operand of O_t += P_t V_j, so P never touches shared memory.
+// P_t (bf16, two per column) overwrites S_t columns [0,32) (keys 0-63) and
+// [64,96) (keys 64-127), each written by the warpgroup that read those scores,
+// and is the TMEM-resident A operand of O_t += P_t V_j, so P never touches
+// shared memory.
 //
 // Per key tile j the MMA thread issues S0 = Q0 K_j^T, S1 = Q1 K_j^T, then
 // O0 += P0 V_j, O1 += P1 V_j as the warpgroups publish P.  S_t of tile j+1 is
@@ -27,12 +30,6 @@
 
 #include "sm100.cuh"
 #include "sigmoid.cuh"
-
-// Which half of a tile's sigma work (0 or 1) hands the MUFU token to the other
-// warpgroup once its last MUFU op is issued.
-#ifndef SIGATTN_FWD_TOKEN_HALF
-#define SIGATTN_FWD_TOKEN_HALF 1
-#endif
 
 namespace sigattn {
 
@@ -61,8 +58,8 @@ struct FwdLayout {
     static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
     // q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2],
-    // pv_done[2], drain, turn[2]
-    static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 9;
+    // drain
+    static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 5;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
     static constexpr int BYTES = OFF_ABORT + 8;
@@ -103,10 +100,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t *v_empty = v_full + VS;
     uint64_t *s_full = v_empty + VS;
     uint64_t *p_full = s_full + 2;
-    uint64_t *pv_done = p_full + 2;
-    uint64_t *drain = pv_done + 2;
-    uint64_t *turn = drain + 1;
-    static_assert(1 + 2 * KS + 2 * VS + 9 == Lay::NBAR, "barrier count");
+    uint64_t *drain = p_full + 2;
+    static_assert(1 + 2 * KS + 2 * VS + 5 == Lay::NBAR, "barrier count");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -137,12 +132,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&s_full[t], 1);
-            mbar_init(&p_full[t], 128);
-            mbar_init(&pv_done[t], 1);
+            mbar_init(&p_full[t], 256);  // both sigma warpgroups
         }
         mbar_init(drain, 1);
-        mbar_init(&turn[0], 128);
-        mbar_init(&turn[1], 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -228,19 +220,20 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 mma_commit(&s_full[t]);
             };
-            // O_t += P_t V_j, P_t read from TMEM (16 keys = 8 packed columns per step)
+            // O_t += P_t V_j, P_t read from TMEM (16 keys = 8 packed columns per step;
+            // keys 64-127 sit 32 columns further on, see the sigma warpgroups)
             auto issue_pv = [&](int t, uint32_t vbase, bool first) {
                 const uint32_t d_tmem = tmem + (t ? Lay::COL_O1 : Lay::COL_O0);
                 const uint32_t a_tmem = tmem + (t ? Lay::COL_S1 : Lay::COL_S0);
 #pragma unroll
                 for (int kk = 0; kk < Lay::BN / 16; ++kk)
-                    mma_ts(d_tmem, a_tmem + kk * 8,
+                    mma_ts(d_tmem, a_tmem + kk * 8 + (kk >= 4 ? 32 : 0),
                            smem_desc_sw128(vbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_o,
                            (!first || kk > 0) ? 1u : 0u);
             };
             // Order per key tile j: PV0_j, S0_{j+1}, PV1_j, S1_{j+1}.  Tile 0's next
-            // scores never wait for tile 1's P, so the two sigma warpgroups can
-            // alternate while the tensor pipe works on the other tile.  S_t of
+            // scores never wait for tile 1's P, so the sigma warps can evaluate
+            // one tile while the tensor pipe works on the other.  S_t of
             // j+1 overwrites P_t of j right after O_t += P_t V_j is issued: MMAs
             // issued by one thread execute in issue order, so the P.V MMA has read
             // P_t before the next scores are written over it.
@@ -279,81 +272,74 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ sigma warpgroups
-        const int t = (warp - 4) >> 2;
+        // Both warpgroups work on every query tile, warpgroup g on key columns
+        // [64 g, 64 g + 64) of S_t, so each sigma phase has two warps per SM
+        // sub-partition: one warp per sub-partition cannot keep the MUFU busy
+        // (its dependent chain leaves issue slots empty).  The tiles alternate:
+        // while the warpgroups evaluate tile t, the tensor pipe runs the other
+        // tile's P.V and next scores.
+        const int g = (warp - 4) >> 2;
         const int quarter = warp & 3;  // TMEM lane quarter this warp may access
-        const int row = (qtile0 + t) * Lay::BM + quarter * 32 + lane;
         const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t tS = tmem + lane_bits + (t ? Lay::COL_S1 : Lay::COL_S0);
-        const uint32_t tO = tmem + lane_bits + (t ? Lay::COL_O1 : Lay::COL_O0);
-        const size_t row_stride = static_cast<size_t>(p.H) * D;
-        __nv_bfloat16 *orow = p.o + (static_cast<size_t>(z) * L + row) * row_stride +
-                              static_cast<size_t>(h) * D;
-        const bool active = work && t < ntiles;
         bool ok = true;
-        if (active) {
+        if (work) {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
-            const bool pingpong = ntiles == 2;
-            for (int j = 0; j < nkv; ++j) {
-                // The two warpgroups take turns (tile 0 first) so that each sigma
-                // phase has the MUFU to itself while the tensor pipe runs the other
-                // tile's P.V and next scores.
-                if (quarter == 0) trace(2 + t, j, 0);
+            // one flat loop over (key tile j, query tile t) steps, t fastest
+            const int nsteps = nkv * ntiles;
+            for (int it = 0; it < nsteps; ++it) {
+                const int t = ntiles == 2 ? (it & 1) : 0;
+                const int j = ntiles == 2 ? (it >> 1) : it;
+                if (quarter == 0) trace(2 + g, j, 2 * t);
                 ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wctx));
                 if (!ok) break;
-                if (quarter == 0) trace(2 + t, j, 1);
-                if (pingpong && (t == 1 || j > 0)) {
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait(&turn[t], (t == 0 ? j - 1 : j) & 1, wctx));
-                    if (!ok) break;
-                }
-                if (quarter == 0) trace(2 + t, j, 2);
+                if (quarter == 0) trace(2 + g, j, 2 * t + 1);
                 tc_fence_after();
-                const int kvalid = nk - j * Lay::BN;   // keys of this tile below n_k
+                const uint32_t tS = tmem + lane_bits + (t ? Lay::COL_S1 : Lay::COL_S0) + 64 * g;
+                uint32_t r[64];
+                tmem_ld64(tS, r);
+                uint32_t pk[32];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    // 64 scores of this row per TMEM read: two exposed load
-                    // latencies per tile
-                    uint32_t r[64];
-                    tmem_ld64(tS + 64 * half, r);
-                    uint32_t pk[32];
+                for (int i = 0; i < 32; ++i) {
+                    const float2 pr = sigma2<MODE>(
+                        scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
+                    pk[i] = pack_bf16x2(pr.x, pr.y);
+                }
+                const int kvalid = nk - j * Lay::BN - 64 * g;  // keys of this half below n_k
+                if (kvalid < 64) {
+                    // last key tile: keys at or beyond n_k weigh exactly zero
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float2 pr = sigma2<MODE>(
-                            scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
-                        pk[i] = pack_bf16x2(pr.x, pr.y);
+                        const uint32_t lo = 2 * i < kvalid ? 0x0000FFFFu : 0u;
+                        const uint32_t hi = 2 * i + 1 < kvalid ? 0xFFFF0000u : 0u;
+                        pk[i] &= (lo | hi);
                     }
-                    // the last MUFU op of this tile is issued: hand the MUFU to the
-                    // other warpgroup before packing and storing
-                    if (half == SIGATTN_FWD_TOKEN_HALF && pingpong) mbar_arrive(&turn[t ^ 1]);
-                    if (kvalid < Lay::BN) {
-                        // last tile: keys at or beyond n_k weigh exactly zero
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int c = 64 * half + 2 * i;
-                            const uint32_t lo = c < kvalid ? 0x0000FFFFu : 0u;
-                            const uint32_t hi = c + 1 < kvalid ? 0xFFFF0000u : 0u;
-                            pk[i] &= (lo | hi);
-                        }
-                    }
-                    // P columns [32 half, 32 half + 32) lie over S columns already read
-                    tmem_st32(tS + 32 * half, pk);
                 }
-                if (quarter == 0) trace(2 + t, j, 3);
+                // P of these 64 keys lies over the first 32 of the S columns
+                // just read; the other warpgroup never touches them
+                tmem_st32(tS, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[t]);
-                if (quarter == 0) trace(2 + t, j, 4);
+                if (quarter == 0) trace(2 + g, j, 4 + t);
             }
             // every MMA of this CTA has finished once the MMA thread's final commit lands
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
+        }
+        // epilogue: warpgroup g writes query tile g
+        const int row = (qtile0 + g) * Lay::BM + quarter * 32 + lane;
+        const size_t row_stride = static_cast<size_t>(p.H) * D;
+        __nv_bfloat16 *orow = p.o + (static_cast<size_t>(z) * L + row) * row_stride +
+                              static_cast<size_t>(h) * D;
+        if (work && g < ntiles) {
             if (ok) {
                 tc_fence_after();
+                const uint32_t tO = tmem + lane_bits + (g ? Lay::COL_O1 : Lay::COL_O0);
                 const bool valid = row < nq;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld32(tO + 32 * c, r);
-                                        if (row < L) {
+                    if (row < L) {
                         uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
 #pragma unroll
                         for (int v4 = 0; v4 < 4; ++v4) {
