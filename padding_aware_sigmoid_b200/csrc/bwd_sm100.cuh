@@ -6,9 +6,10 @@
 //   dQ = alpha dS K,   dK = alpha dS^T Q,   dV = P^T dO.
 //
 // Both kernels share the forward's structure: warps 0 and 2 issue TMA loads
-// (one ring each), one thread of warp 1 issues tcgen05.mma, and two warpgroups (warps 4-7 and
-// 8-11) turn the fp32 score tiles in TMEM into bf16 operands, each owning 64
-// of the 128 columns (thread = TMEM lane = tile row).  The bf16 results are
+// (one ring each), warp 1 issues tcgen05.mma (running converged, one elected
+// lane issuing), and two warpgroups (warps 4-7 and 8-11) turn the fp32 score
+// tiles in TMEM into bf16 operands, each owning 64 of the 128 columns (thread =
+// TMEM lane = tile row).  The bf16 results are
 // written back into TMEM over columns their own warpgroup has already read,
 // and become the TMEM-resident A operand of the next MMA:
 //   warpgroup 0 writes packed columns [base, base+32)     for tile columns 0..63
@@ -251,7 +252,11 @@ __global__ void __launch_bounds__(384, 1)
             ring_drain<SY>(y_full, iy, p.timeout_ns);
         }
     } else if (warp == 1) {
-        if (work && lane == 0) {
+        // the whole warp runs converged; elect.sync picks the issuing lane
+        if (work) {
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, wctx));
+            };
             const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idesc_q = idesc_bf16_f32(128, D, false, true);
             const uint32_t sQ = smem_u32(smem + Lay::OFF_A), sDO = smem_u32(smem + Lay::OFF_B);
@@ -263,52 +268,52 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + col, smem_desc_sw128(xbase + koff, 16, 1024),
-                           smem_desc_sw128(ybase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss_w(tmem + col, smem_desc_sw128(xbase + koff, 16, 1024),
+                             smem_desc_sw128(ybase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            bool ok = mbar_wait(res_full, 0, wctx) && mbar_wait(&x_full[0], 0, wctx) &&
-                      mbar_wait(&y_full[0], 0, wctx);
+            bool ok = wait(res_full, 0) && wait(&x_full[0], 0) && wait(&y_full[0], 0);
             if (ok) {
                 tc_fence_after();
                 issue_xyT(kColS, sQ, kslot(0));
-                mma_commit(s_full);
+                mma_commit_w(s_full);
                 issue_xyT(kColDP0, sDO, vslot(0));
-                mma_commit(&dp_full[0]);
-                mma_commit(&y_empty[0]);
+                mma_commit_w(&dp_full[0]);
+                mma_commit_w(&y_empty[0]);
             }
             for (int j = 0; ok && j < nkv; ++j) {
                 const bool more = j + 1 < nkv;
                 if (more) {
-                    if (!(ok = mbar_wait(&x_full[(j + 1) % SX], ((j + 1) / SX) & 1, wctx))) break;
-                    if (!(ok = mbar_wait(s_free, j & 1, wctx))) break;
-                    trace(1, j, 0);
+                    if (!(ok = wait(&x_full[(j + 1) % SX], ((j + 1) / SX) & 1))) break;
+                    if (!(ok = wait(s_free, j & 1))) break;
+                    if (lane == 0) trace(1, j, 0);
                     tc_fence_after();
                     issue_xyT(kColS, sQ, kslot(j + 1));
-                    mma_commit(s_full);
-                    if (!(ok = mbar_wait(&y_full[(j + 1) % SY], ((j + 1) / SY) & 1, wctx))) break;
+                    mma_commit_w(s_full);
+                    if (!(ok = wait(&y_full[(j + 1) % SY], ((j + 1) / SY) & 1))) break;
                     // buffer (j+1) % 2 still holds dS_{j-1}: dQ += dS_{j-1} K_{j-1} was
                     // issued earlier by this thread and MMAs run in issue order
-                    trace(1, j, 1);
+                    if (lane == 0) trace(1, j, 1);
                     tc_fence_after();
                     issue_xyT((j + 1) & 1 ? kColDP1 : kColDP0, sDO, vslot(j + 1));
-                    mma_commit(&dp_full[(j + 1) & 1]);
-                    mma_commit(&y_empty[(j + 1) % SY]);   // V_{j+1}: its only MMA
+                    mma_commit_w(&dp_full[(j + 1) & 1]);
+                    mma_commit_w(&y_empty[(j + 1) % SY]);  // V_{j+1}: its only MMA
                 }
-                if (!(ok = mbar_wait(&ds_ready[j & 1], (j >> 1) & 1, wctx))) break;
-                trace(1, j, 2);
+                if (!(ok = wait(&ds_ready[j & 1], (j >> 1) & 1))) break;
+                if (lane == 0) trace(1, j, 2);
                 tc_fence_after();
                 const uint32_t dcol = j & 1 ? kColDP1 : kColDP0;
                 const uint32_t sK = kslot(j);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + kColDQ, tmem + dcol + packed_col(kk),
-                           smem_desc_sw128(sK + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_q,
-                           (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&x_empty[j % SX]);             // K_j: S_j and dQ_j done
+                    mma_ts_w(tmem + kColDQ, tmem + dcol + packed_col(kk),
+                             smem_desc_sw128(sK + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_q,
+                             (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit_w(&x_empty[j % SX]);           // K_j: S_j and dQ_j done
             }
-            mma_commit(drain);
+            mma_commit_w(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
+            __syncwarp();
         }
     } else if (warp >= 4) {
         const int w = (warp - 4) >> 2;      // warpgroup: tile columns [64w, 64w+64)
@@ -501,7 +506,11 @@ __global__ void __launch_bounds__(384, 1)
             ring_drain<SY>(y_full, iy, p.timeout_ns);
         }
     } else if (warp == 1) {
-        if (work && lane == 0) {
+        // the whole warp runs converged; elect.sync picks the issuing lane
+        if (work) {
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, wctx));
+            };
             const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idesc_kv = idesc_bf16_f32(128, D, false, true);
             const uint32_t sK = smem_u32(smem + Lay::OFF_A), sV = smem_u32(smem + Lay::OFF_B);
@@ -512,59 +521,59 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                    mma_ss(tmem + col, smem_desc_sw128(xbase + koff, 16, 1024),
-                           smem_desc_sw128(ybase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss_w(tmem + col, smem_desc_sw128(xbase + koff, 16, 1024),
+                             smem_desc_sw128(ybase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // acc += A(TMEM, packed over `acol`) * B (128 query rows, MN-major)
             auto issue_acc = [&](uint32_t acc, uint32_t acol, uint32_t bbase, bool first) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + acc, tmem + acol + packed_col(kk),
-                           smem_desc_sw128(bbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_kv,
-                           (!first || kk > 0) ? 1u : 0u);
+                    mma_ts_w(tmem + acc, tmem + acol + packed_col(kk),
+                             smem_desc_sw128(bbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_kv,
+                             (!first || kk > 0) ? 1u : 0u);
             };
-            bool ok = mbar_wait(res_full, 0, wctx) && mbar_wait(&x_full[0], 0, wctx) &&
-                      mbar_wait(&y_full[0], 0, wctx);
+            bool ok = wait(res_full, 0) && wait(&x_full[0], 0) && wait(&y_full[0], 0);
             if (ok) {
                 tc_fence_after();
                 issue_xyT(Lay::COL_S, sK, qslot(0));
-                mma_commit(s_full);
+                mma_commit_w(s_full);
                 issue_xyT(Lay::COL_DP, sV, doslot(0));
-                mma_commit(dp_full);
+                mma_commit_w(dp_full);
             }
             for (int i = 0; ok && i < nqt; ++i) {
                 const bool more = i + 1 < nqt;
-                if (!(ok = mbar_wait(p_ready, i & 1, wctx))) break;
-                trace(1, i, 0);
+                if (!(ok = wait(p_ready, i & 1))) break;
+                if (lane == 0) trace(1, i, 0);
                 tc_fence_after();
                 issue_acc(Lay::COL_ACC0, Lay::COL_S, doslot(i), i == 0);      // dV += P^T dO_i
-                mma_commit(&y_empty[i % SY]);                                 // dO_i: dP^T_i, dV_i done
+                mma_commit_w(&y_empty[i % SY]);                                 // dO_i: dP^T_i, dV_i done
                 if (more) {
                     // S^T_{i+1} overwrites P^T_i, read by the dV MMA just issued
                     // (MMAs run in issue order)
-                    if (!(ok = mbar_wait(&x_full[(i + 1) % SX], ((i + 1) / SX) & 1, wctx))) break;
-                    trace(1, i, 1);
+                    if (!(ok = wait(&x_full[(i + 1) % SX], ((i + 1) / SX) & 1))) break;
+                    if (lane == 0) trace(1, i, 1);
                     tc_fence_after();
                     issue_xyT(Lay::COL_S, sK, qslot(i + 1));
-                    mma_commit(s_full);
+                    mma_commit_w(s_full);
                 }
-                if (!(ok = mbar_wait(ds_ready, i & 1, wctx))) break;
-                trace(1, i, 2);
+                if (!(ok = wait(ds_ready, i & 1))) break;
+                if (lane == 0) trace(1, i, 2);
                 tc_fence_after();
                 issue_acc(Lay::COL_ACC1, Lay::COL_DP, qslot(i), i == 0);      // dK += dS^T Q_i
-                mma_commit(&x_empty[i % SX]);                                 // Q_i: S^T_i, dK_i done
+                mma_commit_w(&x_empty[i % SX]);                                 // Q_i: S^T_i, dK_i done
                 if (more) {
                     // dP^T_{i+1} overwrites dS^T_i, read by the dK MMA just issued
-                    if (!(ok = mbar_wait(&y_full[(i + 1) % SY], ((i + 1) / SY) & 1, wctx))) break;
-                    trace(1, i, 3);
+                    if (!(ok = wait(&y_full[(i + 1) % SY], ((i + 1) / SY) & 1))) break;
+                    if (lane == 0) trace(1, i, 3);
                     tc_fence_after();
                     issue_xyT(Lay::COL_DP, sV, doslot(i + 1));
-                    mma_commit(dp_full);
+                    mma_commit_w(dp_full);
                 }
             }
-            mma_commit(drain);
+            mma_commit_w(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
+            __syncwarp();
         }
     } else if (warp >= 4) {
         const int w = (warp - 4) >> 2;      // warpgroup: query columns [64w, 64w+64)
