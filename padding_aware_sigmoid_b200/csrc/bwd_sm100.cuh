@@ -393,12 +393,17 @@ __global__ void __launch_bounds__(384, 1)
 // Works on the transposed scores (rows = keys):
 //   S^T = K Q_i^T, dP^T = V dO_i^T, P^T -> TMEM over S^T, dS^T -> TMEM over dP^T,
 //   dV += P^T dO_i, dK += dS^T Q_i.
-// TMEM: [0,128) S^T / P^T, [128,256) dP^T / dS^T, [256,256+D) dV, [256+D,256+2D) dK.
+// TMEM: [0,128) S^T, [128,256) dP^T, then P^T and dS^T over it,
+// [256,256+D) dV, [256+D,256+2D) dK.
 //
-// The warpgroups publish P^T first (it needs S^T only) and dS^T second; the
-// MMA order per query tile is dV_i, S^T_{i+1} (over P^T_i, which dV_i has read:
-// MMAs from one thread run in issue order), dK_i, dP^T_{i+1} (over dS^T_i), so
-// the sigma work on i+1 overlaps dK_i.
+// A warpgroup reads its 64 columns of S^T into registers and releases the S^T
+// buffer at once, so S^T_{i+1} is computed while it evaluates sigma and
+// sigma' for tile i.  It keeps P^T in registers until it has read its dP^T
+// columns, then writes P^T over the first 32 of them (tile columns 64w..64w+63
+// packed two per column) and dS^T over the other 32.  MMA order per query
+// tile: S^T_{i+1} (as soon as S^T_i is read), dV_i, dK_i, dP^T_{i+1} (over P^T_i
+// and dS^T_i, read by dV_i and dK_i just before: MMAs from one thread run in
+// issue order).
 // ============================================================================
 template <int D, int MODE, int SX, int SY>
 __global__ void __launch_bounds__(384, 1)
@@ -416,12 +421,11 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t *y_empty = y_full + SY;
     uint64_t *s_full = y_empty + SY;          // MMA -> WGs: S^T_i in TMEM
     uint64_t *dp_full = s_full + 1;           // MMA -> WGs: dP^T_i in TMEM
-    uint64_t *p_ready = dp_full + 1;          // WGs -> MMA: P^T_i in TMEM
+    uint64_t *s_free = dp_full + 1;           // WGs -> MMA: S^T_i read
+    uint64_t *p_ready = s_free + 1;           // WGs -> MMA: P^T_i in TMEM
     uint64_t *ds_ready = p_ready + 1;         // WGs -> MMA: dS^T_i in TMEM
-    uint64_t *dv_done = ds_ready + 1;         // MMA: dV += P^T_i dO_i finished
-    uint64_t *dk_done = dv_done + 1;          // MMA: dK += dS^T_i Q_i finished
-    uint64_t *drain = dk_done + 1;
-    static_assert(7 <= Lay::MAX_HANDOFF, "barrier count");
+    uint64_t *drain = ds_ready + 1;
+    static_assert(6 <= Lay::MAX_HANDOFF, "barrier count");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -449,10 +453,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
+        mbar_init(s_free, 256);
         mbar_init(p_ready, 256);
         mbar_init(ds_ready, 256);
-        mbar_init(dv_done, 1);
-        mbar_init(dk_done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -543,27 +546,28 @@ __global__ void __launch_bounds__(384, 1)
             }
             for (int i = 0; ok && i < nqt; ++i) {
                 const bool more = i + 1 < nqt;
-                if (!(ok = wait(p_ready, i & 1))) break;
-                if (lane == 0) trace(1, i, 0);
-                tc_fence_after();
-                issue_acc(Lay::COL_ACC0, Lay::COL_S, doslot(i), i == 0);      // dV += P^T dO_i
-                mma_commit_w(&y_empty[i % SY]);                                 // dO_i: dP^T_i, dV_i done
                 if (more) {
-                    // S^T_{i+1} overwrites P^T_i, read by the dV MMA just issued
-                    // (MMAs run in issue order)
+                    // S^T_{i+1} into the S^T buffer as soon as the warpgroups have read S^T_i
                     if (!(ok = wait(&x_full[(i + 1) % SX], ((i + 1) / SX) & 1))) break;
-                    if (lane == 0) trace(1, i, 1);
+                    if (!(ok = wait(s_free, i & 1))) break;
+                    if (lane == 0) trace(1, i, 0);
                     tc_fence_after();
                     issue_xyT(Lay::COL_S, sK, qslot(i + 1));
                     mma_commit_w(s_full);
                 }
+                if (!(ok = wait(p_ready, i & 1))) break;
+                if (lane == 0) trace(1, i, 1);
+                tc_fence_after();
+                issue_acc(Lay::COL_ACC0, Lay::COL_DP, doslot(i), i == 0);       // dV += P^T dO_i
+                mma_commit_w(&y_empty[i % SY]);                                 // dO_i: dP^T_i, dV_i done
                 if (!(ok = wait(ds_ready, i & 1))) break;
                 if (lane == 0) trace(1, i, 2);
                 tc_fence_after();
-                issue_acc(Lay::COL_ACC1, Lay::COL_DP, qslot(i), i == 0);      // dK += dS^T Q_i
+                issue_acc(Lay::COL_ACC1, Lay::COL_DP + 32, qslot(i), i == 0);  // dK += dS^T Q_i
                 mma_commit_w(&x_empty[i % SX]);                                 // Q_i: S^T_i, dK_i done
                 if (more) {
-                    // dP^T_{i+1} overwrites dS^T_i, read by the dK MMA just issued
+                    // dP^T_{i+1} overwrites P^T_i and dS^T_i, read by the two MMAs just
+                    // issued (MMAs run in issue order)
                     if (!(ok = wait(&y_full[(i + 1) % SY], ((i + 1) / SY) & 1))) break;
                     if (lane == 0) trace(1, i, 3);
                     tc_fence_after();
@@ -586,18 +590,23 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         if (work) {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
+            const uint32_t tS = tmem + lane_bits + Lay::COL_S + 64 * w;
+            const uint32_t tD = tmem + lane_bits + Lay::COL_DP + 64 * w;
             for (int i = 0; i < nqt; ++i) {
                 const int qvalid = nq - i * 128;
                 float2 g[32];
+                uint32_t pk[32];
+                if (quarter == 0) trace(2 + w, i, 0);
+                ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
+                if (!ok) break;
+                if (quarter == 0) trace(2 + w, i, 1);
+                tc_fence_after();
                 {
-                    if (quarter == 0) trace(2 + w, i, 0);
-                    ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
-                    if (!ok) break;
-                    if (quarter == 0) trace(2 + w, i, 1);
-                    tc_fence_after();
                     uint32_t r[64];
-                    tmem_ld64(tmem + lane_bits + Lay::COL_S + 64 * w, r);
-                    uint32_t pk[32];
+                    tmem_ld64(tS, r);
+                    // S^T_i is in registers: the MMA warp may compute S^T_{i+1} now
+                    tc_fence_before();
+                    mbar_arrive(s_free);
 #pragma unroll
                     for (int ii = 0; ii < 32; ++ii) {
                         float2 pr;
@@ -605,27 +614,40 @@ __global__ void __launch_bounds__(384, 1)
                                           pr, g[ii]);
                         pk[ii] = pack_bf16x2(pr.x, pr.y);
                     }
-                    if (qvalid < 128) mask_packed(pk, 64 * w, qvalid);
-                    tmem_st32(tmem + lane_bits + Lay::COL_S + 64 * w, pk);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(p_ready);
-                    if (quarter == 0) trace(2 + w, i, 2);
                 }
+                if (qvalid < 128) mask_packed(pk, 64 * w, qvalid);
+                if (quarter == 0) trace(2 + w, i, 2);
                 ok = __all_sync(0xffffffffu, mbar_wait(dp_full, i & 1, wctx));
                 if (!ok) break;
                 if (quarter == 0) trace(2 + w, i, 3);
                 tc_fence_after();
-                uint32_t d[64];
-                tmem_ld64(tmem + lane_bits + Lay::COL_DP + 64 * w, d);
-                uint32_t pk[32];
+                uint32_t ds[32];
+                {
+                    // first 32 dP^T columns, then P^T over them
+                    uint32_t d[32];
+                    tmem_ld32(tD, d);
+                    tmem_st32(tD, pk);
 #pragma unroll
-                for (int ii = 0; ii < 32; ++ii) {
-                    const float2 ds = mul2(g[ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
-                    pk[ii] = pack_bf16x2(ds.x, ds.y);
+                    for (int ii = 0; ii < 16; ++ii) {
+                        const float2 v = mul2(g[ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
+                        ds[ii] = pack_bf16x2(v.x, v.y);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(p_ready);
                 }
-                if (qvalid < 128) mask_packed(pk, 64 * w, qvalid);
-                tmem_st32(tmem + lane_bits + Lay::COL_DP + 64 * w, pk);
+                {
+                    // the other 32 dP^T columns, then dS^T over them
+                    uint32_t d[32];
+                    tmem_ld32(tD + 32, d);
+#pragma unroll
+                    for (int ii = 0; ii < 16; ++ii) {
+                        const float2 v = mul2(g[16 + ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
+                        ds[16 + ii] = pack_bf16x2(v.x, v.y);
+                    }
+                }
+                if (qvalid < 128) mask_packed(ds, 64 * w, qvalid);
+                tmem_st32(tD + 32, ds);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ds_ready);
