@@ -419,13 +419,27 @@ def our_arm(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def kernel_source_hash() -> str:
+    """sha256 over the CUDA sources of the library (file names and contents)."""
+    import hashlib
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "padding_aware_sigmoid_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        h.update(name.encode())
+        with open(os.path.join(src, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def _ncu_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary of the same kernel, if
-    one exists for the current build; None otherwise."""
+    """DRAM bytes per launch from the committed ncu capture of the same kernel,
+    or None when there is none or the kernel sources changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
+        if d.get("_meta", {}).get("source_sha256") != kernel_source_hash():
+            return None
         return d.get(kernel)
     except Exception:
         return None
