@@ -104,6 +104,17 @@ def _p(a: np.ndarray, ct):
     return a.ctypes.data_as(ctypes.POINTER(ct))
 
 
+def _bias(bias, Z: int) -> np.ndarray:
+    """The bias as one float64 per sample: a scalar is broadcast to every sample."""
+    b = np.asarray(bias, dtype=np.float64)
+    if b.ndim == 0:
+        return np.full(Z, float(b), dtype=np.float64)
+    b = np.ascontiguousarray(b.reshape(-1))
+    if b.shape[0] != Z:
+        raise ValueError(f"bias has {b.shape[0]} entries, expected {Z}")
+    return b
+
+
 class OracleLib:
     """One loaded build of the oracle.  The module-level functions use the
     default build; tests may load a deliberately altered copy to show that the
@@ -118,12 +129,14 @@ class OracleLib:
         lib.oracle_sigmoid.restype = cd
         lib.oracle_sigmoid_grad.argtypes = [cd]
         lib.oracle_sigmoid_grad.restype = cd
-        lib.oracle_fwd_rows.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd, cd,
+        lib.oracle_fwd_rows.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
                                         i64p, c64, f64p]
-        lib.oracle_dq_rows.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd, cd,
+        lib.oracle_dq_rows.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
                                        i64p, c64, f64p]
         lib.oracle_dkdv_rows.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd,
-                                         cd, i64p, c64, f64p, f64p]
+                                         f64p, i64p, c64, f64p, f64p]
+        lib.oracle_dbias.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
+                                     f64p, f64p]
         lib.oracle_num_threads.restype = ci
         self.lib = lib
         self.path = path
@@ -144,9 +157,10 @@ class OracleLib:
         qa, ka, va, _, dt, (Z, L, H, D), nq, nk = _common(q, k, v, None, seqlens_q, seqlens_k)
         it = _items(items)
         out = np.zeros((it.shape[0], D), dtype=np.float64)
+        bz = _bias(bias, Z)
         self.lib.oracle_fwd_rows(_vp(qa), _vp(ka), _vp(va), dt, Z, L, H, D,
                                  _p(nq, ctypes.c_int32), _p(nk, ctypes.c_int32),
-                                 float(alpha), float(bias), _p(it, ctypes.c_int64),
+                                 float(alpha), _p(bz, ctypes.c_double), _p(it, ctypes.c_int64),
                                  it.shape[0], _p(out, ctypes.c_double))
         return out
 
@@ -155,9 +169,10 @@ class OracleLib:
         qa, ka, va, da, dt, (Z, L, H, D), nq, nk = _common(q, k, v, dout, seqlens_q, seqlens_k)
         it = _items(items)
         out = np.zeros((it.shape[0], D), dtype=np.float64)
+        bz = _bias(bias, Z)
         self.lib.oracle_dq_rows(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, L, H, D,
                                 _p(nq, ctypes.c_int32), _p(nk, ctypes.c_int32),
-                                float(alpha), float(bias), _p(it, ctypes.c_int64),
+                                float(alpha), _p(bz, ctypes.c_double), _p(it, ctypes.c_int64),
                                 it.shape[0], _p(out, ctypes.c_double))
         return out
 
@@ -167,9 +182,10 @@ class OracleLib:
         it = _items(items)
         dk = np.zeros((it.shape[0], D), dtype=np.float64)
         dv = np.zeros((it.shape[0], D), dtype=np.float64)
+        bz = _bias(bias, Z)
         self.lib.oracle_dkdv_rows(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, L, H, D,
                                   _p(nq, ctypes.c_int32), _p(nk, ctypes.c_int32),
-                                  float(alpha), float(bias), _p(it, ctypes.c_int64),
+                                  float(alpha), _p(bz, ctypes.c_double), _p(it, ctypes.c_int64),
                                   it.shape[0], _p(dk, ctypes.c_double), _p(dv, ctypes.c_double))
         return dk, dv
 
@@ -178,6 +194,20 @@ class OracleLib:
         Z, L, H, D = (int(s) for s in q.shape)
         rows = self.fwd_rows(q, k, v, seqlens_q, seqlens_k, alpha, bias, all_rows(Z, L, H))
         return rows.reshape(Z, L, H, D)
+
+    def dbias(self, q, k, v, dout, seqlens_q, seqlens_k, alpha, bias) -> np.ndarray:
+        """Bias gradient per sample, float64 [Z]: db_z = sum over heads and valid
+        (i, j) of dS_ij (paperlayer.ai summary, section 3; gist.science summary,
+        section 2.A: x = alpha q.k + b, so dx/db = 1)."""
+        qa, ka, va, da, dt, (Z, L, H, D), nq, nk = _common(q, k, v, dout, seqlens_q, seqlens_k)
+        bz = _bias(bias, Z)
+        rowsum = np.zeros(Z * H * L, dtype=np.float64)
+        out = np.zeros(Z, dtype=np.float64)
+        self.lib.oracle_dbias(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, L, H, D,
+                              _p(nq, ctypes.c_int32), _p(nk, ctypes.c_int32), float(alpha),
+                              _p(bz, ctypes.c_double), _p(rowsum, ctypes.c_double),
+                              _p(out, ctypes.c_double))
+        return out
 
     def bwd(self, q, k, v, dout, seqlens_q, seqlens_k, alpha, bias):
         """Full backward (dQ, dK, dV) as float64 [Z, L, H, D] each."""
@@ -225,6 +255,10 @@ def dq_rows(*a, **kw):
 
 def dkdv_rows(*a, **kw):
     return default().dkdv_rows(*a, **kw)
+
+
+def dbias(*a, **kw):
+    return default().dbias(*a, **kw)
 
 
 def fwd(*a, **kw):

@@ -20,6 +20,11 @@
  *       dQ = alpha dS K; dK/dV by the transposed view: dK = alpha dS^T Q,
  *       dV = P^T dO.  Padded query rows are constants (written as zero), so no
  *       gradient flows from them: their dO is ignored.
+ *   paperlayer.ai summary, section 3 (background on sigmoid attention) and
+ *       gist.science summary, section 2.A (bias term): the bias is set to
+ *       b = -log(n); here b may differ per sample (bias_z[z], e.g. -ln n_z),
+ *       and since x_ij = alpha q_i.k_j + b_z, the gradient of a per-sample
+ *       bias is db_z = sum over heads and valid (i, j) of dS_ij.
  *
  * Readings where the pages are silent are listed in the design notes; here:
  *   - the -inf mask is applied by selection (P = 0), never by adding -inf;
@@ -29,6 +34,7 @@
  * Layout of every tensor: [Z][L][H][D], contiguous; element (z,l,h,d) sits at
  * ((z*L + l)*H + h)*D + d.  dtype 0 = bf16 (raw uint16 bits), 1 = fp32.
  * Row lists are int64 triples (z, h, row).  Outputs are double, D per row.
+ * bias_z holds one bias per sample (double[Z]).
  *
  * Parallelism: OpenMP over independent rows only; each row is summed in
  * ascending index order, exactly as the definition reads.
@@ -89,7 +95,7 @@ static int clamp_len(int n, int L) { return n < 0 ? 0 : (n > L ? L : n); }
 /* Forward rows: O[z, i, h, :] = [i < n_q] sum_{j < n_k} sigma(x_ij) V[z, j, h, :]. */
 void oracle_fwd_rows(const void *q, const void *k, const void *v, int dtype,
                      int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
-                     double alpha, double bias, const int64_t *items, int64_t nitems,
+                     double alpha, const double *bias_z, const int64_t *items, int64_t nitems,
                      double *out) {
     (void)Z;
 #pragma omp parallel for schedule(dynamic, 4)
@@ -98,6 +104,7 @@ void oracle_fwd_rows(const void *q, const void *k, const void *v, int dtype,
         double *o = out + t * D;
         for (int d = 0; d < D; ++d) o[d] = 0.0;
         int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        const double bias = bias_z[z];
         if (i >= n_q) continue;
         for (int64_t j = 0; j < n_k; ++j) {
             double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
@@ -111,7 +118,7 @@ void oracle_fwd_rows(const void *q, const void *k, const void *v, int dtype,
  * dS_ij = P_ij (1 - P_ij) (dO_i . V_j). */
 void oracle_dq_rows(const void *q, const void *k, const void *v, const void *dout, int dtype,
                     int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
-                    double alpha, double bias, const int64_t *items, int64_t nitems,
+                    double alpha, const double *bias_z, const int64_t *items, int64_t nitems,
                     double *out) {
     (void)Z;
 #pragma omp parallel for schedule(dynamic, 4)
@@ -120,6 +127,7 @@ void oracle_dq_rows(const void *q, const void *k, const void *v, const void *dou
         double *g = out + t * D;
         for (int d = 0; d < D; ++d) g[d] = 0.0;
         int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        const double bias = bias_z[z];
         if (i >= n_q) continue;
         for (int64_t j = 0; j < n_k; ++j) {
             double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
@@ -137,7 +145,7 @@ void oracle_dq_rows(const void *q, const void *k, const void *v, const void *dou
  *   dK[z, j, h, :] = [j < n_k] alpha sum_{i < n_q} dS_ij Q[z, i, h, :] */
 void oracle_dkdv_rows(const void *q, const void *k, const void *v, const void *dout, int dtype,
                       int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
-                      double alpha, double bias, const int64_t *items, int64_t nitems,
+                      double alpha, const double *bias_z, const int64_t *items, int64_t nitems,
                       double *dk_out, double *dv_out) {
     (void)Z;
 #pragma omp parallel for schedule(dynamic, 4)
@@ -146,6 +154,7 @@ void oracle_dkdv_rows(const void *q, const void *k, const void *v, const void *d
         double *gk = dk_out + t * D, *gv = dv_out + t * D;
         for (int d = 0; d < D; ++d) { gk[d] = 0.0; gv[d] = 0.0; }
         int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        const double bias = bias_z[z];
         if (j >= n_k) continue;
         for (int64_t i = 0; i < n_q; ++i) {
             double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
@@ -158,6 +167,36 @@ void oracle_dkdv_rows(const void *q, const void *k, const void *v, const void *d
             }
         }
         for (int d = 0; d < D; ++d) gk[d] *= alpha;
+    }
+}
+
+/* Bias gradient per sample: db_z = sum_h sum_{i < n_q} sum_{j < n_k} dS_ij with
+ * dS_ij = P_ij (1 - P_ij) (dO_i . V_j).  One partial per (z, h, i) row, each summed
+ * in ascending j; the partials are then added in ascending (h, i) order per
+ * sample, so the result does not depend on the thread count. */
+void oracle_dbias(const void *q, const void *k, const void *v, const void *dout, int dtype,
+                  int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
+                  double alpha, const double *bias_z, double *rowsum, double *dbias) {
+    const int64_t nrows = (int64_t)Z * H * L;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t t = 0; t < nrows; ++t) {
+        int64_t z = t / ((int64_t)H * L), h = (t / L) % H, i = t % L;
+        double acc = 0.0;
+        int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        const double bias = bias_z[z];
+        if (i < n_q) {
+            for (int64_t j = 0; j < n_k; ++j) {
+                double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
+                double dp = dot_rows(dout, v, dtype, z, h, i, j, L, H, D);
+                acc += p * (1.0 - p) * dp;
+            }
+        }
+        rowsum[t] = acc;
+    }
+    for (int64_t z = 0; z < Z; ++z) {
+        double s = 0.0;
+        for (int64_t r = 0; r < (int64_t)H * L; ++r) s += rowsum[z * H * L + r];
+        dbias[z] = s;
     }
 }
 

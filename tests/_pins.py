@@ -13,7 +13,10 @@ mathematics fix:
 * closed-form special cases (alpha = 0, a single valid key);
 * invariants (padding never changes results, padded rows are zero, linearity in
   V, permutation equivariance, the two bilinearity identities of the gradients);
-* central finite differences of the oracle's own (pinned) forward.
+* central finite differences of the oracle's own (pinned) forward;
+* a per-sample bias (paperlayer.ai summary, section 3: b = -log(n)) and its
+  gradient db against torch autograd, the alpha = 0 closed form and a finite
+  difference.
 
 ``tests/test_oracle_pins.py`` runs them on the real oracle and
 ``tests/test_oracle_mutants.py`` shows that builds with one plausible mistake
@@ -327,6 +330,89 @@ def pin_bf16_widening_and_rows(orc):
         _close(rows[t], b[z, i, h], 0, 0, "row subset indexing")
 
 
+# ---------------------------------------------------------------- per-sample bias, db
+
+
+def pin_per_sample_bias_autograd(orc):
+    """Per-sample bias b_z (paperlayer.ai summary, section 3: b = -log(n) per
+    sequence) and its gradient db_z = sum dS, against torch fp64 autograd with b
+    as a leaf tensor."""
+    for seed, kw in [(160, {}), (170, dict(Z=3, L=6, H=2, D=3, nq=(6, 0, 3), nk=(4, 6, 6))),
+                     (180, dict(Z=2, L=5, H=3, D=4, nq=(5, 2), nk=(2, 5), scale=3.0))]:
+        q, k, v, do, nq, nk = _case(seed, **kw)
+        Z, L, H, D = q.shape
+        alpha = 0.45
+        bz = -np.log(np.maximum(nk, 1).astype(np.float64)) + 0.1 * np.arange(Z)
+        tq, tk, tv = (torch.tensor(a.astype(np.float64), requires_grad=True) for a in (q, k, v))
+        tb = torch.tensor(bz, requires_grad=True)
+        tdo = torch.from_numpy(do.astype(np.float64))
+        kmask = torch.zeros((Z, L), dtype=torch.float64)
+        qmask = torch.zeros((Z, L), dtype=torch.float64)
+        for z in range(Z):
+            kmask[z, : nk[z]] = 1.0
+            qmask[z, : nq[z]] = 1.0
+        s = alpha * torch.einsum("zihd,zjhd->zhij", tq, tk) + tb[:, None, None, None]
+        p = torch.sigmoid(s) * kmask[:, None, None, :]
+        o = torch.einsum("zhij,zjhd->zihd", p, tv) * qmask[:, :, None, None]
+        (o * tdo).sum().backward()
+        _close(orc.fwd(q, k, v, nq, nk, alpha, bz), o.detach().numpy(), 1e-12, 1e-13,
+               f"forward with per-sample bias vs torch (seed {seed})")
+        dq, dk, dv = orc.bwd(q, k, v, do, nq, nk, alpha, bz)
+        _close(dq, tq.grad.numpy(), 1e-11, 1e-12, f"dQ with per-sample bias (seed {seed})")
+        _close(dk, tk.grad.numpy(), 1e-11, 1e-12, f"dK with per-sample bias (seed {seed})")
+        _close(dv, tv.grad.numpy(), 1e-11, 1e-12, f"dV with per-sample bias (seed {seed})")
+        _close(orc.dbias(q, k, v, do, nq, nk, alpha, bz), tb.grad.numpy(), 1e-11, 1e-12,
+               f"db vs torch autograd (seed {seed})")
+
+
+def pin_per_sample_bias_slices(orc):
+    """A per-sample bias equals running each sample alone with its scalar bias."""
+    q, k, v, do, nq, nk = _case(190, Z=3, L=6, H=2, D=3, nq=(6, 3, 1), nk=(5, 6, 2))
+    alpha, bz = 0.6, np.array([-1.2, 0.4, -2.5])
+    o = orc.fwd(q, k, v, nq, nk, alpha, bz)
+    g = orc.bwd(q, k, v, do, nq, nk, alpha, bz)
+    db = orc.dbias(q, k, v, do, nq, nk, alpha, bz)
+    for z in range(3):
+        sl = slice(z, z + 1)
+        args = (q[sl], k[sl], v[sl])
+        lens = (nq[sl], nk[sl], alpha, float(bz[z]))
+        _close(o[sl], orc.fwd(*args, *lens), 0, 0, "per-sample bias: forward slice")
+        for x, y in zip(g, orc.bwd(*args, do[sl], *lens)):
+            _close(x[sl], y, 0, 0, "per-sample bias: gradient slice")
+        _close(db[z], orc.dbias(*args, do[sl], *lens)[0], 0, 0, "per-sample bias: db slice")
+
+
+def pin_dbias_alpha_zero(orc):
+    """alpha = 0: every valid score is b_z, so dS_ij = sigma'(b_z) dO_i.V_j and
+    db_z = sigma'(b_z) sum_h (sum_{i<n_q} dO_i) . (sum_{j<n_k} V_j)."""
+    q, k, v, do, nq, nk = _case(200, Z=2, L=7, H=3, D=4, nq=(7, 3), nk=(2, 7))
+    bz = np.array([-0.7, 1.1])
+    db = orc.dbias(q, k, v, do, nq, nk, 0.0, bz)
+    for z in range(2):
+        s = _sigma_tanh(bz[z])
+        dosum = do[z, : nq[z]].astype(np.float64).sum(axis=0)   # [H, D]
+        vsum = v[z, : nk[z]].astype(np.float64).sum(axis=0)     # [H, D]
+        _close(db[z], s * (1 - s) * float(np.sum(dosum * vsum)), 1e-12, 1e-13,
+               "alpha=0: db closed form")
+
+
+def pin_dbias_finite_difference(orc):
+    """db_z against a central difference of sum(O * dO) in b_z."""
+    q, k, v, do, nq, nk = _case(210, Z=2, L=6, H=2, D=3, nq=(5, 6), nk=(6, 3))
+    alpha, bz = 0.8, np.array([-1.5, -0.4])
+    db = orc.dbias(q, k, v, do, nq, nk, alpha, bz)
+    do64 = do.astype(np.float64)
+    h = 2.0 ** -12
+    for z in range(2):
+        bp, bm = bz.copy(), bz.copy()
+        bp[z] += h
+        bm[z] -= h
+        fd = (np.sum(orc.fwd(q, k, v, nq, nk, alpha, bp) * do64) -
+              np.sum(orc.fwd(q, k, v, nq, nk, alpha, bm) * do64)) / (2 * h)
+        if abs(fd - db[z]) > 1e-7 * max(1.0, abs(db[z])):
+            raise AssertionError(f"db[{z}]: oracle {db[z]} vs finite difference {fd}")
+
+
 ALL_PINS = [
     pin_sigmoid_closed_forms,
     pin_sigmoid_derivative,
@@ -341,4 +427,8 @@ ALL_PINS = [
     pin_gradient_identities,
     pin_finite_differences,
     pin_bf16_widening_and_rows,
+    pin_per_sample_bias_autograd,
+    pin_per_sample_bias_slices,
+    pin_dbias_alpha_zero,
+    pin_dbias_finite_difference,
 ]

@@ -37,6 +37,10 @@ MUTANTS = [
     ("dkdv-no-key-row-mask", "if (j >= n_k) continue;", "", None),
     ("layout-h-l-swapped", "return ((z * L + l) * H + h) * (int64_t)D;",
      "return ((z * H + h) * L + l) * (int64_t)D;", None),
+    ("dbias-dropped-sigma-prime", "acc += p * (1.0 - p) * dp;", "acc += p * dp;", None),
+    ("dbias-no-key-mask", "for (int64_t j = 0; j < n_k; ++j) {", "for (int64_t j = 0; j < L; ++j) {", 2),
+    ("dbias-no-query-mask", "if (i < n_q) {", "if (i < L) {", None),
+    ("bias-per-sample-wrong-index", "const double bias = bias_z[z];", "const double bias = bias_z[0];", None),
     ("bf16-widening", "uint32_t bits = ((uint32_t)b) << 16;", "uint32_t bits = ((uint32_t)b) << 15;", None),
     ("fwd-value-from-key", "for (int d = 0; d < D; ++d) o[d] += p * load_elem(v, dtype, vo + d);",
      "for (int d = 0; d < D; ++d) o[d] += p * load_elem(k, dtype, vo + d);", None),
