@@ -44,6 +44,7 @@
 #ifndef SIGATTN_H
 #define SIGATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -116,6 +117,43 @@ sigattn_status sigattn_bwd_dkdv(const void *q, const void *k, const void *v, con
                                 void *dk, void *dv, const int32_t *seqlens_q,
                                 const int32_t *seqlens_k, int Z, int L, int H, int D,
                                 float alpha, float bias, sigattn_dtype dtype, void *stream);
+
+/* Per-sample bias and its gradient.
+ *
+ * The pages set the bias to b = -log(n) (paperlayer.ai summary, section 3,
+ * background on sigmoid attention; gist.science summary, section 2.A, bias
+ * term) and note that this choice was never swept (paper.rainbus.top summary,
+ * limitations).  These calls take one bias per sample, so b_z = -ln n_z or a
+ * learned value can be used, and return the bias gradient
+ *     db_z = sum over heads h and valid (i < n_q, j < n_k) of dS_zhij,
+ * since x = alpha q.k + b_z.  For one bias shared by all samples, sum db over z.
+ *
+ * sigattn_fwd_bias: as sigattn_fwd, with `bias` a device float[Z] (not NULL
+ * when Z > 0) in place of the scalar.
+ *
+ * sigattn_bwd_bias: as sigattn_bwd, with `bias` a device float[Z].  `dbias`,
+ * if not NULL, is a device float[Z] that receives db; it is computed from the
+ * fp32 dS values of the dQ pass, summed per dQ work unit and then per sample
+ * in a fixed order (the result does not depend on scheduling).  That needs a
+ * caller-owned device `workspace` of at least
+ * sigattn_dbias_workspace_bytes(Z, L, H, dtype) bytes, 4-byte aligned, which
+ * the call overwrites (its contents on entry do not matter).  With dbias NULL
+ * the workspace is not used and may be NULL.
+ * Errors: SIGATTN_ERR_INVALID_ARG when bias is NULL, or dbias is set and the
+ * workspace is missing, too small or misaligned; otherwise as sigattn_bwd. */
+sigattn_status sigattn_fwd_bias(const void *q, const void *k, const void *v, void *o,
+                                const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int L,
+                                int H, int D, float alpha, const float *bias, sigattn_dtype dtype,
+                                void *stream);
+sigattn_status sigattn_bwd_bias(const void *q, const void *k, const void *v, const void *dout,
+                                void *dq, void *dk, void *dv, const int32_t *seqlens_q,
+                                const int32_t *seqlens_k, int Z, int L, int H, int D, float alpha,
+                                const float *bias, float *dbias, void *workspace,
+                                size_t workspace_bytes, sigattn_dtype dtype, void *stream);
+/* Bytes of device workspace sigattn_bwd_bias needs to return dbias (0 for an
+ * empty problem): one float per dQ work unit (bf16: per 128-row query tile
+ * and head; fp32: per query row and head) of every sample. */
+size_t sigattn_dbias_workspace_bytes(int Z, int L, int H, sigattn_dtype dtype);
 
 /* Selects how later bf16 calls in this process evaluate sigma (process-wide,
  * default SIGATTN_SIGMOID_TANH, the pages' form; see sigattn_sigmoid_mode).  Returns

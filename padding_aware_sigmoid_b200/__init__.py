@@ -22,6 +22,7 @@ __all__ = [
     "last_device_status", "set_wait_timeout_ns", "selftest_wait_timeout", "status_string",
     "version", "library_path", "load_library", "SIGMOID_TANH", "SIGMOID_EXP", "EXPORTS",
     "SigmoidAttention", "bwd_dq", "bwd_dkdv", "last_cuda_error", "fwd_noalloc", "NOALLOC_MAX_Z",
+    "fwd_bias", "bwd_bias", "dbias_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -48,7 +49,7 @@ EXPORTS = (
     "sigattn_set_sigmoid_mode", "sigattn_get_sigmoid_mode", "sigattn_sigmoid_eval",
     "sigattn_last_device_status", "sigattn_set_wait_timeout_ns", "sigattn_selftest_wait_timeout",
     "sigattn_last_cuda_error", "sigattn_status_string", "sigattn_version",
-    "sigattn_fwd_noalloc",
+    "sigattn_fwd_noalloc", "sigattn_fwd_bias", "sigattn_bwd_bias", "sigattn_dbias_workspace_bytes",
 )
 
 
@@ -85,6 +86,13 @@ def load_library():
         lib.sigattn_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf,
                                          ci, vp]
         lib.sigattn_bwd_dkdv.restype = ci
+        lib.sigattn_fwd_bias.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, vp, ci, vp]
+        lib.sigattn_fwd_bias.restype = ci
+        lib.sigattn_bwd_bias.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf,
+                                         vp, vp, vp, ctypes.c_size_t, ci, vp]
+        lib.sigattn_bwd_bias.restype = ci
+        lib.sigattn_dbias_workspace_bytes.argtypes = [ci, ci, ci, ci]
+        lib.sigattn_dbias_workspace_bytes.restype = ctypes.c_size_t
         lib.sigattn_last_cuda_error.restype = ctypes.c_char_p
         lib.sigattn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf, ci, vp]
         lib.sigattn_fwd_noalloc.restype = ci
@@ -205,6 +213,67 @@ def bwd_dkdv(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, dk=
         seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, L, H, D, float(alpha), float(bias),
         _dtype_code(q), _stream_ptr(q)), "sigattn_bwd_dkdv")
     return dk, dv
+
+
+def _check_bias(bias, ref):
+    import torch
+    if not (bias.is_cuda and bias.dtype == torch.float32 and bias.dim() == 1 and
+            bias.shape[0] == ref.shape[0] and bias.is_contiguous() and bias.device == ref.device):
+        raise ValueError("bias must be a contiguous float32 [Z] tensor on the tensors' device")
+
+
+def fwd_bias(q, k, v, seqlens_q, seqlens_k, alpha: float, bias, out=None):
+    """Forward with one bias per sample: ``bias`` is a float32 [Z] CUDA tensor
+    (for example -log(n_z)); otherwise as ``fwd``."""
+    import torch
+    _check_inputs([q, k, v], [seqlens_q, seqlens_k])
+    _check_bias(bias, q)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_inputs([q, out], [])
+    Z, L, H, D = (int(s) for s in q.shape)
+    _check(load_library().sigattn_fwd_bias(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), seqlens_q.data_ptr(),
+        seqlens_k.data_ptr(), Z, L, H, D, float(alpha), bias.data_ptr(), _dtype_code(q),
+        _stream_ptr(q)), "sigattn_fwd_bias")
+    return out
+
+
+def dbias_workspace_bytes(Z: int, L: int, H: int, dtype) -> int:
+    """Device workspace bytes ``bwd_bias`` needs to return the bias gradient."""
+    import torch
+    code = _FP32 if dtype == torch.float32 else _BF16
+    return int(load_library().sigattn_dbias_workspace_bytes(int(Z), int(L), int(H), code))
+
+
+def bwd_bias(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias, want_dbias: bool = True,
+             dq=None, dk=None, dv=None, workspace=None):
+    """(dQ, dK, dV, db) with one bias per sample (``bias``: float32 [Z] CUDA
+    tensor); db[z] = sum over heads and valid (i, j) of dS (None when
+    ``want_dbias`` is false).  The db workspace is allocated here unless given."""
+    import torch
+    _check_inputs([q, k, v, dout], [seqlens_q, seqlens_k])
+    _check_bias(bias, q)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_inputs([q, dq, dk, dv], [])
+    Z, L, H, D = (int(s) for s in q.shape)
+    db = None
+    ws_ptr, ws_bytes = None, 0
+    if want_dbias:
+        db = torch.empty(Z, dtype=torch.float32, device=q.device)
+        need = dbias_workspace_bytes(Z, L, H, q.dtype)
+        if workspace is None:
+            workspace = torch.empty(max(need // 4, 1), dtype=torch.float32, device=q.device)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    _check(load_library().sigattn_bwd_bias(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+        dv.data_ptr(), seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, L, H, D, float(alpha),
+        bias.data_ptr(), None if db is None else db.data_ptr(), ws_ptr, ws_bytes,
+        _dtype_code(q), _stream_ptr(q)), "sigattn_bwd_bias")
+    return dq, dk, dv, db
 
 
 def fwd_noalloc(q, k, v, seqlens_q, seqlens_k, alpha: float, bias: float, out=None):

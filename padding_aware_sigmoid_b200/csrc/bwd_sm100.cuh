@@ -37,6 +37,8 @@ struct BwdParams {
     float alpha, bias;
     int *status;
     uint64_t timeout_ns;
+    const float *bias_z;   // device float[Z], one bias per sample; null: the scalar `bias`
+    float *db_part;        // dQ kernel: one partial of db_z = sum dS per CTA, or null
 };
 
 // Shared memory: two resident tiles (dq: Q, dO; dkdv: K, V) and two rings of
@@ -60,7 +62,8 @@ struct BwdLayout {
     static constexpr int NBAR = 1 + 2 * SX + 2 * SY + MAX_HANDOFF;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
-    static constexpr int SMEM_ALLOC = OFF_ABORT + 8 + 1024;
+    static constexpr int OFF_RED = OFF_ABORT + 8;      // 8 floats: per-warp db partials
+    static constexpr int SMEM_ALLOC = OFF_RED + 32 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
     static_assert(COL_ACC1 + D <= TMEM_COLS, "TMEM budget");
@@ -323,8 +326,10 @@ __global__ void __launch_bounds__(384, 1)
         __nv_bfloat16 *drow = p.dq + (static_cast<size_t>(z) * L + row) * (static_cast<size_t>(p.H) * D) +
                               static_cast<size_t>(h) * D;
         bool ok = true;
+        const bool want_db = p.db_part != nullptr;
+        float dbacc = 0.0f;   // bias gradient: sum of this row's dS (valid rows and keys)
         if (work) {
-            const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
+            const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             for (int j = 0; j < nkv; ++j) {
                 float2 g[32];
                 {
@@ -355,12 +360,19 @@ __global__ void __launch_bounds__(384, 1)
                 tmem_ld64(tmem + lane_bits + dcol, d);
                 if (quarter == 0) trace(2 + w, j, 5);
                 uint32_t pk[32];
+                const int kvalid = nk - j * 128;
+                float2 dsum = f2(0.0f, 0.0f);   // this row's fp32 dS over keys below n_k
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float2 ds = mul2(g[i], f2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
                     pk[i] = pack_bf16x2(ds.x, ds.y);
+                    if (want_db) {
+                        const int c = 64 * w + 2 * i;
+                        dsum.x += c < kvalid ? ds.x : 0.0f;
+                        dsum.y += c + 1 < kvalid ? ds.y : 0.0f;
+                    }
                 }
-                const int kvalid = nk - j * 128;
+                dbacc += dsum.x + dsum.y;
                 if (kvalid < 128) mask_packed(pk, 64 * w, kvalid);
                 tmem_st32(tmem + lane_bits + dcol, pk);
                 tmem_wait_st();
@@ -377,6 +389,21 @@ __global__ void __launch_bounds__(384, 1)
             }
         } else if (row < L) {
             zero_row<D>(drow, w * (D / 2), D / 2);
+        }
+        if (want_db) {
+            // one partial per CTA, summed in a fixed order: warp sums, then the
+            // eight warps' sums in warp order (rows at or beyond n_q add nothing)
+            float v = row < nq ? dbacc : 0.0f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            float *red = reinterpret_cast<float *>(smem + Lay::OFF_RED);
+            if (lane == 0) red[warp - 4] = v;
+            sigma_warps_sync(256);
+            if (warp == 4 && lane == 0) {
+                float t = 0.0f;
+                for (int u = 0; u < 8; ++u) t += red[u];
+                p.db_part[(static_cast<size_t>(z) * p.H + h) * gridDim.x + qtile] = t;
+            }
         }
     }
 
@@ -589,7 +616,7 @@ __global__ void __launch_bounds__(384, 1)
         __nv_bfloat16 *dst = (w == 0 ? p.dv : p.dk) + roff;
         bool ok = true;
         if (work) {
-            const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
+            const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             const uint32_t tS = tmem + lane_bits + Lay::COL_S + 64 * w;
             const uint32_t tD = tmem + lane_bits + Lay::COL_DP + 64 * w;
             for (int i = 0; i < nqt; ++i) {
@@ -671,6 +698,23 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         tmem_dealloc(tmem, Lay::TMEM_COLS);
     }
+}
+
+// db_z = sum of the per-CTA (or per-row) partials of sample z, in double and in
+// a fixed order: thread t adds partials t, t + 256, ...; then a fixed tree.
+__global__ void __launch_bounds__(256) dbias_reduce_kernel(const float *part, int64_t per_z,
+                                                           float *dbias) {
+    __shared__ double red[256];
+    const int z = blockIdx.x;
+    double acc = 0.0;
+    for (int64_t t = threadIdx.x; t < per_z; t += 256) acc += part[z * per_z + t];
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int s = 128; s > 0; s >>= 1) {
+        if (static_cast<int>(threadIdx.x) < s) red[threadIdx.x] += red[threadIdx.x + s];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) dbias[z] = static_cast<float>(red[0]);
 }
 
 }  // namespace sigattn

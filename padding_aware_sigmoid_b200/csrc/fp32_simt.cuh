@@ -33,6 +33,8 @@ struct F32Params {
     int Z, L, H;
     float alpha, bias;
     int *status;
+    const float *bias_z;   // device float[Z], one bias per sample; null: the scalar `bias`
+    float *db_part;        // dQ kernel: sum of dS per row ([Z][L][H] order), or null
 };
 
 __device__ __forceinline__ void clamp_lengths(const F32Params &p, int z, int &nq, int &nk) {
@@ -58,6 +60,7 @@ __global__ void __launch_bounds__(256) f32_fwd_kernel(const F32Params p) {
     const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.L));
     int nq, nk;
     clamp_lengths(p, z, nq, nk);
+    const float bias = bias_of(p.bias_z, p.bias, z);
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.0f;
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(256) f32_fwd_kernel(const F32Params p) {
             for (int e = 0; e < E; ++e) s = fmaf(qv[e], p.k[kr * D + lane + 32 * e], s);
             s = warp_sum(s);
             float pr, g;
-            exact_sigma(fmaf(p.alpha, s, p.bias), pr, g);
+            exact_sigma(fmaf(p.alpha, s, bias), pr, g);
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[e] = fmaf(pr, p.v[kr * D + lane + 32 * e], acc[e]);
         }
@@ -93,9 +96,11 @@ __global__ void __launch_bounds__(256) f32_dq_kernel(const F32Params p) {
     const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.L));
     int nq, nk;
     clamp_lengths(p, z, nq, nk);
+    const float bias = bias_of(p.bias_z, p.bias, z);
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+    float dbacc = 0.0f;   // sum of this row's dS over keys below n_k
     if (i < nq) {
         float qv[E], gv[E];
 #pragma unroll
@@ -114,14 +119,16 @@ __global__ void __launch_bounds__(256) f32_dq_kernel(const F32Params p) {
             s = warp_sum(s);
             dp = warp_sum(dp);
             float pr, g;
-            exact_sigma(fmaf(p.alpha, s, p.bias), pr, g);
+            exact_sigma(fmaf(p.alpha, s, bias), pr, g);
             const float ds = g * dp;
+            dbacc += ds;
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[e] = fmaf(ds, p.k[kr * D + lane + 32 * e], acc[e]);
         }
     }
 #pragma unroll
     for (int e = 0; e < E; ++e) p.dq[r * D + lane + 32 * e] = p.alpha * acc[e];
+    if (p.db_part != nullptr && lane == 0) p.db_part[r] = dbacc;
 }
 
 template <int D>
@@ -136,6 +143,7 @@ __global__ void __launch_bounds__(256) f32_dkdv_kernel(const F32Params p) {
     const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.L));
     int nq, nk;
     clamp_lengths(p, z, nq, nk);
+    const float bias = bias_of(p.bias_z, p.bias, z);
     float ak[E], av[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) ak[e] = av[e] = 0.0f;
@@ -157,7 +165,7 @@ __global__ void __launch_bounds__(256) f32_dkdv_kernel(const F32Params p) {
             s = warp_sum(s);
             dp = warp_sum(dp);
             float pr, g;
-            exact_sigma(fmaf(p.alpha, s, p.bias), pr, g);
+            exact_sigma(fmaf(p.alpha, s, bias), pr, g);
             const float ds = g * dp;
 #pragma unroll
             for (int e = 0; e < E; ++e) {

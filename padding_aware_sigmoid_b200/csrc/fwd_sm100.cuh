@@ -41,6 +41,7 @@ struct FwdParams {
     float alpha, bias;
     int *status;
     uint64_t timeout_ns;
+    const float *bias_z;   // device float[Z], one bias per sample; null: the scalar `bias`
 };
 
 // Shared memory: the two query tiles, a ring of KS key tiles and a ring of VS
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
         bool ok = true;
         if (work) {
-            const SigmoidCoef cf = make_coef<MODE>(p.alpha, p.bias);
+            const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             // one flat loop over (key tile j, query tile t) steps, t fastest
             const int nsteps = nkv * ntiles;
             for (int it = 0; it < nsteps; ++it) {

@@ -157,11 +157,20 @@ sigattn_status bwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
     return SIGATTN_OK;
 }
 
-// Shared body of sigattn_bwd, sigattn_bwd_dq and sigattn_bwd_dkdv.
+// Partials of db per sample: one per dQ CTA (bf16) or per query row (fp32).
+int64_t dbias_partials_per_sample(int L, int H, sigattn_dtype dtype) {
+    return dtype == SIGATTN_FP32 ? static_cast<int64_t>(L) * H
+                                 : static_cast<int64_t>((L + 127) / 128) * H;
+}
+
+// Shared body of sigattn_bwd, sigattn_bwd_dq, sigattn_bwd_dkdv and sigattn_bwd_bias.
+// bias_z (device float[Z]) replaces the scalar bias when not null; dbias (device
+// float[Z]) receives the bias gradient when not null, through `work`.
 sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void *dout, void *dq,
                         void *dk, void *dv, const int32_t *seqlens_q, const int32_t *seqlens_k,
                         int Z, int L, int H, int D, float alpha, float bias, sigattn_dtype dtype,
-                        void *stream, int parts) {
+                        void *stream, int parts, const float *bias_z = nullptr,
+                        float *dbias = nullptr, float *work = nullptr) {
     bool empty = false;
     sigattn_status s = check_shape(Z, L, H, D, dtype, &empty);
     if (s != SIGATTN_OK) return s;
@@ -169,6 +178,8 @@ sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void 
     if (!q || !k || !v || !dout || !seqlens_q || !seqlens_k) return SIGATTN_ERR_INVALID_ARG;
     if (((parts & kPartDq) && !dq) || ((parts & kPartDkdv) && (!dk || !dv)))
         return SIGATTN_ERR_INVALID_ARG;
+    if (dbias && (!work || !(parts & kPartDq))) return SIGATTN_ERR_INVALID_ARG;
+    float *db_part = dbias ? work : nullptr;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
         ((parts & kPartDq) && !aligned16(dq)) ||
         ((parts & kPartDkdv) && (!aligned16(dk) || !aligned16(dv))))
@@ -183,7 +194,7 @@ sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void 
                     nullptr,                          static_cast<float *>(dq),
                     static_cast<float *>(dk),         static_cast<float *>(dv),
                     seqlens_q,                        seqlens_k,
-                    Z, L, H, alpha, bias, status};
+                    Z, L, H, alpha, bias, status, bias_z, db_part};
         const int64_t rows = static_cast<int64_t>(Z) * L * H;
         dim3 grid(static_cast<unsigned>((rows + 7) / 8));
         if (parts & kPartDq) {
@@ -191,9 +202,14 @@ sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void 
                         : launch(f32_dq_kernel<128>, grid, dim3(256), 0, st, p);
             if (s != SIGATTN_OK) return s;
         }
-        if (parts & kPartDkdv)
-            return D == 64 ? launch(f32_dkdv_kernel<64>, grid, dim3(256), 0, st, p)
-                           : launch(f32_dkdv_kernel<128>, grid, dim3(256), 0, st, p);
+        if (parts & kPartDkdv) {
+            s = D == 64 ? launch(f32_dkdv_kernel<64>, grid, dim3(256), 0, st, p)
+                        : launch(f32_dkdv_kernel<128>, grid, dim3(256), 0, st, p);
+            if (s != SIGATTN_OK) return s;
+        }
+        if (dbias)
+            return launch(dbias_reduce_kernel, dim3(Z), dim3(256), 0, st, static_cast<const float *>(db_part),
+                          dbias_partials_per_sample(L, H, dtype), dbias);
         return SIGATTN_OK;
     }
     if (cc != 100) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
@@ -205,23 +221,24 @@ sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void 
     if ((s = encode_bf16_map(&mdo, dout, Z, L, H, D)) != SIGATTN_OK) return s;
     BwdParams p{static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
                 static_cast<__nv_bfloat16 *>(dv), seqlens_q, seqlens_k, L, H, alpha, bias, status,
-                g_timeout_ns.load()};
+                g_timeout_ns.load(), bias_z, db_part};
     const int mode = g_sigmoid_mode.load();
     if (D == 128)
-        return mode == kSigmoidTanh
-                   ? bwd_bf16<128, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, L, H, parts, st)
-                   : bwd_bf16<128, kSigmoidExp>(mq, mk, mv, mdo, p, Z, L, H, parts, st);
-    return mode == kSigmoidTanh ? bwd_bf16<64, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, L, H, parts, st)
-                                : bwd_bf16<64, kSigmoidExp>(mq, mk, mv, mdo, p, Z, L, H, parts, st);
+        s = mode == kSigmoidTanh ? bwd_bf16<128, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, L, H, parts, st)
+                                 : bwd_bf16<128, kSigmoidExp>(mq, mk, mv, mdo, p, Z, L, H, parts, st);
+    else
+        s = mode == kSigmoidTanh ? bwd_bf16<64, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, L, H, parts, st)
+                                 : bwd_bf16<64, kSigmoidExp>(mq, mk, mv, mdo, p, Z, L, H, parts, st);
+    if (s != SIGATTN_OK || !dbias) return s;
+    return launch(dbias_reduce_kernel, dim3(Z), dim3(256), 0, st, static_cast<const float *>(db_part),
+                  dbias_partials_per_sample(L, H, dtype), dbias);
 }
 
-}  // namespace
-
-extern "C" {
-
-sigattn_status sigattn_fwd(const void *q, const void *k, const void *v, void *o,
-                           const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int L, int H,
-                           int D, float alpha, float bias, sigattn_dtype dtype, void *stream) {
+// Shared body of sigattn_fwd and sigattn_fwd_bias.
+sigattn_status fwd_impl(const void *q, const void *k, const void *v, void *o,
+                        const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int L, int H,
+                        int D, float alpha, float bias, const float *bias_z, sigattn_dtype dtype,
+                        void *stream) {
     bool empty = false;
     sigattn_status s = check_shape(Z, L, H, D, dtype, &empty);
     if (s != SIGATTN_OK) return s;
@@ -236,7 +253,8 @@ sigattn_status sigattn_fwd(const void *q, const void *k, const void *v, void *o,
     if (dtype == SIGATTN_FP32) {
         F32Params p{static_cast<const float *>(q), static_cast<const float *>(k),
                     static_cast<const float *>(v), nullptr, static_cast<float *>(o), nullptr,
-                    nullptr, nullptr, seqlens_q, seqlens_k, Z, L, H, alpha, bias, status};
+                    nullptr, nullptr, seqlens_q, seqlens_k, Z, L, H, alpha, bias, status,
+                    bias_z, nullptr};
         const int64_t rows = static_cast<int64_t>(Z) * L * H;
         dim3 grid(static_cast<unsigned>((rows + 7) / 8));
         return D == 64 ? launch(f32_fwd_kernel<64>, grid, dim3(256), 0, st, p)
@@ -249,13 +267,53 @@ sigattn_status sigattn_fwd(const void *q, const void *k, const void *v, void *o,
     if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
     if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
     FwdParams p{static_cast<__nv_bfloat16 *>(o), seqlens_q, seqlens_k, L, H, alpha, bias, status,
-                g_timeout_ns.load()};
+                g_timeout_ns.load(), bias_z};
     const int mode = g_sigmoid_mode.load();
     if (D == 128)
         return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
                                     : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
     return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
                                 : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+sigattn_status sigattn_fwd(const void *q, const void *k, const void *v, void *o,
+                           const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int L, int H,
+                           int D, float alpha, float bias, sigattn_dtype dtype, void *stream) {
+    return fwd_impl(q, k, v, o, seqlens_q, seqlens_k, Z, L, H, D, alpha, bias, nullptr, dtype,
+                    stream);
+}
+
+sigattn_status sigattn_fwd_bias(const void *q, const void *k, const void *v, void *o,
+                                const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int L,
+                                int H, int D, float alpha, const float *bias, sigattn_dtype dtype,
+                                void *stream) {
+    if (!bias && Z > 0) return SIGATTN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, o, seqlens_q, seqlens_k, Z, L, H, D, alpha, 0.0f, bias, dtype, stream);
+}
+
+size_t sigattn_dbias_workspace_bytes(int Z, int L, int H, sigattn_dtype dtype) {
+    if (Z <= 0 || L <= 0 || H <= 0) return 0;
+    return static_cast<size_t>(Z) * static_cast<size_t>(dbias_partials_per_sample(L, H, dtype)) *
+           sizeof(float);
+}
+
+sigattn_status sigattn_bwd_bias(const void *q, const void *k, const void *v, const void *dout,
+                                void *dq, void *dk, void *dv, const int32_t *seqlens_q,
+                                const int32_t *seqlens_k, int Z, int L, int H, int D, float alpha,
+                                const float *bias, float *dbias, void *workspace,
+                                size_t workspace_bytes, sigattn_dtype dtype, void *stream) {
+    if (!bias && Z > 0) return SIGATTN_ERR_INVALID_ARG;
+    if (dbias && Z > 0 && L > 0 && H > 0) {
+        if (!workspace || workspace_bytes < sigattn_dbias_workspace_bytes(Z, L, H, dtype) ||
+            (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+            return SIGATTN_ERR_INVALID_ARG;
+    }
+    return bwd_impl(q, k, v, dout, dq, dk, dv, seqlens_q, seqlens_k, Z, L, H, D, alpha, 0.0f, dtype,
+                    stream, kPartDq | kPartDkdv, bias, dbias, static_cast<float *>(workspace));
 }
 
 sigattn_status sigattn_bwd(const void *q, const void *k, const void *v, const void *dout, void *dq,
@@ -450,7 +508,7 @@ sigattn_status sigattn_fwd_noalloc(const void *q, const void *k, const void *v, 
     if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
     if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
     FwdParams p{static_cast<__nv_bfloat16 *>(o), nq, nk, L, H, alpha, bias, status,
-                g_timeout_ns.load()};
+                g_timeout_ns.load(), nullptr};
     const int mode = g_sigmoid_mode.load();
     if (D == 128)
         return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)

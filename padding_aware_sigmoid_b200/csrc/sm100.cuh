@@ -342,6 +342,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Bias of sample z: one value per sample when the caller passes an array
+// (e.g. b_z = -ln n_z), otherwise the scalar.
+__device__ __forceinline__ float bias_of(const float *bias_z, float bias, int z) {
+    return bias_z != nullptr ? bias_z[z] : bias;
+}
+
+// Named barrier 1 over the `count` threads of the sigma warpgroups.
+__device__ __forceinline__ void sigma_warps_sync(int count) {
+    asm volatile("bar.sync 1, %0;" ::"r"(count) : "memory");
+}
+
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 

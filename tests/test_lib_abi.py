@@ -81,6 +81,32 @@ def test_host_validation_needs_no_gpu(lib):
     assert lib.sigattn_set_wait_timeout_ns(0) == 1
 
 
+def test_bias_entry_points_host_validation(lib):
+    import padding_aware_sigmoid_b200 as sa
+    vp = ctypes.c_void_p
+    dummy = vp(16)
+    # workspace: one float per dQ work unit (bf16: 128-row query tile x head; fp32: row x head)
+    assert sa.dbias_workspace_bytes(2, 300, 3, __import__("torch").bfloat16) == 2 * 3 * 3 * 4
+    assert sa.dbias_workspace_bytes(2, 300, 3, __import__("torch").float32) == 2 * 300 * 3 * 4
+    assert lib.sigattn_dbias_workspace_bytes(0, 128, 1, 0) == 0
+    # a null bias array is rejected before any device call
+    assert lib.sigattn_fwd_bias(dummy, dummy, dummy, dummy, dummy, dummy, 1, 128, 1, 64, 1.0,
+                                None, 0, None) == 1
+    assert lib.sigattn_bwd_bias(dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                128, 1, 64, 1.0, None, None, None, 0, 0, None) == 1
+    # dbias requested without a large enough, aligned workspace
+    need = lib.sigattn_dbias_workspace_bytes(1, 128, 1, 0)
+    assert lib.sigattn_bwd_bias(dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                128, 1, 64, 1.0, dummy, dummy, None, need, 0, None) == 1
+    assert lib.sigattn_bwd_bias(dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                128, 1, 64, 1.0, dummy, dummy, dummy, need - 4, 0, None) == 1
+    assert lib.sigattn_bwd_bias(dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                128, 1, 64, 1.0, dummy, dummy, vp(16 + 2), need, 0, None) == 1
+    # empty problems are a no-op
+    assert lib.sigattn_fwd_bias(dummy, dummy, dummy, dummy, dummy, dummy, 0, 128, 1, 64, 1.0,
+                                None, 0, None) == 0
+
+
 def test_no_cpu_fallback(lib):
     import torch
     import padding_aware_sigmoid_b200 as sa
