@@ -149,7 +149,8 @@ __device__ __forceinline__ void mask_packed(uint32_t (&pk)[32], int col0, int va
 // warpgroups run their sigma' phase at the same time, so that two warps share
 // each SM sub-partition's MUFU (one warp alone leaves it idle between issues).
 // ============================================================================
-template <int D, int MODE, int SX, int SY>
+// DB: also accumulate the bias gradient (p.db_part must then be set)
+template <int D, int MODE, int SX, int SY, bool DB>
 __global__ void __launch_bounds__(384, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -326,7 +327,6 @@ __global__ void __launch_bounds__(384, 1)
         __nv_bfloat16 *drow = p.dq + (static_cast<size_t>(z) * L + row) * (static_cast<size_t>(p.H) * D) +
                               static_cast<size_t>(h) * D;
         bool ok = true;
-        const bool want_db = p.db_part != nullptr;
         float dbacc = 0.0f;   // bias gradient: sum of this row's dS (valid rows and keys)
         if (work) {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
@@ -366,13 +366,13 @@ __global__ void __launch_bounds__(384, 1)
                 for (int i = 0; i < 32; ++i) {
                     const float2 ds = mul2(g[i], f2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
                     pk[i] = pack_bf16x2(ds.x, ds.y);
-                    if (want_db) {
+                    if constexpr (DB) {
                         const int c = 64 * w + 2 * i;
                         dsum.x += c < kvalid ? ds.x : 0.0f;
                         dsum.y += c + 1 < kvalid ? ds.y : 0.0f;
                     }
                 }
-                dbacc += dsum.x + dsum.y;
+                if constexpr (DB) dbacc += dsum.x + dsum.y;
                 if (kvalid < 128) mask_packed(pk, 64 * w, kvalid);
                 tmem_st32(tmem + lane_bits + dcol, pk);
                 tmem_wait_st();
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(384, 1)
         } else if (row < L) {
             zero_row<D>(drow, w * (D / 2), D / 2);
         }
-        if (want_db) {
+        if constexpr (DB) {
             // one partial per CTA, summed in a fixed order: warp sums, then the
             // eight warps' sums in warp order (rows at or beyond n_q add nothing)
             float v = row < nq ? dbacc : 0.0f;

@@ -147,8 +147,12 @@ sigattn_status bwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
     constexpr int SX = BwdStages<D>::X, SY = BwdStages<D>::Y;
     constexpr size_t smem = BwdLayout<D, SX, SY>::SMEM_ALLOC;
     if (parts & kPartDq) {
-        sigattn_status s = launch(bwd_dq_kernel<D, MODE, SX, SY>, grid, dim3(384), smem, st, mq,
-                                  mk, mv, mdo, p);
+        sigattn_status s =
+            p.db_part != nullptr
+                ? launch(bwd_dq_kernel<D, MODE, SX, SY, true>, grid, dim3(384), smem, st, mq, mk,
+                         mv, mdo, p)
+                : launch(bwd_dq_kernel<D, MODE, SX, SY, false>, grid, dim3(384), smem, st, mq, mk,
+                         mv, mdo, p);
         if (s != SIGATTN_OK) return s;
     }
     if (parts & kPartDkdv)

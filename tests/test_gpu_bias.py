@@ -240,3 +240,33 @@ def test_bias_workload_sampled(index):
         valid = C.valid_row_mask(items, n)
         assert np.all(got[~valid] == 0.0)
         C.assert_close(got[valid], ref[valid], "bf16", name)
+
+
+def test_autograd_learnable_and_per_sample_bias():
+    """The module's bias options through autograd: a learnable scalar b gets
+    sum_z db_z, and per-sample b_z = -ln n_k(z) matches the oracle."""
+    dev = _dev()
+    Z, L, H, D = 2, 256, 2, 64
+    q, k, v, do, nq, nk, _ = _inputs(Z, L, H, D, (256, 100), (256, 100), seed=3400)
+    alpha = 1.0 / math.sqrt(D)
+    nqd, nkd = torch.as_tensor(nq, device=dev), torch.as_tensor(nk, device=dev)
+    # learnable scalar
+    mod = sa.SigmoidAttention(bias=-1.5, learnable_bias=True).to(dev)
+    tq, tk, tv = (t.to(dev).clone().requires_grad_(True) for t in (q, k, v))
+    o = mod(tq, tk, tv, nqd, nkd)
+    o.backward(do.to(dev))
+    torch.cuda.synchronize()
+    bz = np.full(Z, -1.5, np.float32)
+    rdb = oracle.dbias(q, k, v, do, nq, nk, alpha, bz).sum()
+    scale = _abs_ds_sum(q, k, v, do, nq, nk, alpha, bz).sum()
+    assert abs(mod.b.grad.item() - rdb) <= DB_TOL["tanh"] * scale
+    rdq, rdk, rdv = oracle.bwd(q, k, v, do, nq, nk, alpha, bz)
+    C.assert_close(tq.grad.float().cpu().numpy(), rdq, "bf16", "dQ (learnable bias)")
+    C.assert_close(tv.grad.float().cpu().numpy(), rdv, "bf16", "dV (learnable bias)")
+    # per-sample -ln n_k
+    mod2 = sa.SigmoidAttention(per_sample_bias=True)
+    o2 = mod2(q.to(dev), k.to(dev), v.to(dev), nqd, nkd)
+    torch.cuda.synchronize()
+    bz2 = (-np.log(nk.astype(np.float64))).astype(np.float32)
+    C.assert_close(o2.float().cpu().numpy(), oracle.fwd(q, k, v, nq, nk, alpha, bz2), "bf16",
+                   "O (per-sample -ln n)")
