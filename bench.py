@@ -336,6 +336,25 @@ def our_arm(args, world, rank, local):
     del inp4
     torch.cuda.empty_cache()
 
+    # the D = 64 workloads (2: short ragged sequences, 5: lognormal lengths, large
+    # scores), timed the same way with their own valid-FLOP counts
+    d64 = {}
+    for idx in (2, 5):
+        w = W.WORKLOADS[idx]
+        inp = make_device_inputs(w, device, rank)
+        st_ms, f_ms, q_ms, kv_ms = time_workload(sa, w, inp, max(args.steps // 2, 3),
+                                                 args.warmup, device)
+        fl = W.fwd_flops_valid(W.lengths(w), W.lengths(w), w.H, w.D)
+        d64[w.name] = {
+            "fwd_tflops": fl / (f_ms * 1e-3) / 1e12,
+            "bwd_tflops": 2.5 * fl / ((q_ms + kv_ms) * 1e-3) / 1e12,
+            "fwd_ms": f_ms, "bwd_dq_ms": q_ms, "bwd_dkdv_ms": kv_ms,
+            "valid_fraction_of_padded_flops":
+                fl / W.fwd_flops_padded(w.Z, w.L, w.H, w.D),
+        }
+        del inp
+    torch.cuda.empty_cache()
+
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_workload(sa, w3, max(args.steps // 4, 3), 2, device)
@@ -404,6 +423,7 @@ def our_arm(args, world, rank, local):
             "bwd_padding_loss_pct": 100.0 * (1.0 - bwd4_tf / bwd_tf),
             "ms_per_step": step4_ms,
         },
+        "workloads_d64": d64,
         "roofline": {
             "kernel": dom, "bound": "tensor", "achieved": achieved, "peak": pk["bf16"],
             "unit": "TFLOP/s", "frac": achieved / pk["bf16"], "traffic": traffic,
@@ -412,7 +432,7 @@ def our_arm(args, world, rank, local):
             "flops_per_launch": dom_flops,
         },
         "clocks": clk.summary(),
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 3 * args.steps,   # the timed headline steps: fwd, dQ, dK/dV
         "e2e": e2e,
         "cpu_baseline": cpu,
     }
