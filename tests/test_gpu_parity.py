@@ -242,3 +242,18 @@ def test_autograd_module_matches_oracle():
     torch.cuda.synchronize()
     _check_full(inp, (o.detach(), q.grad, k.grad, v.grad), "bf16")
 
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_long_sequence_sampled(D):
+    """L = 65536 (4x the headline length) with one full and one ragged sample:
+    sampled rows of every output against the oracle (index arithmetic beyond
+    2^31 elements per tensor row range, deepest loops)."""
+    dev = _dev()
+    Z, L, H = 2, 65536, 1
+    n = (65536, 40001)
+    inp = _case(Z, L, H, D, n, n, seed=4000 + D)
+    outs = _run(inp, dev)
+    rep = _check_sampled(inp, outs, 12, seed=40 + D)
+    print(f"L=65536 D={D}: max-abs/max|ref| / L1 rel:",
+          {k: ("%.2e/%.2e" % v) for k, v in rep.items()})
