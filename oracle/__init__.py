@@ -80,16 +80,20 @@ def _common(q, k, v, dout, seqlens_q, seqlens_k):
         da, dt_o = _as_raw(dout)
         if dt_o != dt:
             raise TypeError("dout must share the dtype of q")
-    if qa.ndim != 4 or qa.shape != ka.shape or qa.shape != va.shape:
-        raise ValueError("q, k, v must be [Z, L, H, D] of one shape")
+    # q (and dout) are [Z, Lq, H, D]; k and v are [Z, Lk, H, D]
+    if qa.ndim != 4 or ka.ndim != 4 or ka.shape != va.shape:
+        raise ValueError("q, k, v must be [Z, L, H, D]; k and v of one shape")
+    if qa.shape[0] != ka.shape[0] or qa.shape[2:] != ka.shape[2:]:
+        raise ValueError("q and k must agree in Z, H and D")
     if da is not None and da.shape != qa.shape:
         raise ValueError("dout must match q's shape")
-    Z, L, H, D = (int(s) for s in qa.shape)
+    Z, Lq, H, D = (int(s) for s in qa.shape)
+    Lk = int(ka.shape[1])
     nq = np.ascontiguousarray(np.asarray(seqlens_q, dtype=np.int32).reshape(-1))
     nk = np.ascontiguousarray(np.asarray(seqlens_k, dtype=np.int32).reshape(-1))
     if nq.shape[0] != Z or nk.shape[0] != Z:
         raise ValueError("seqlens must have Z entries")
-    return qa, ka, va, da, dt, (Z, L, H, D), nq, nk
+    return qa, ka, va, da, dt, (Z, Lq, Lk, H, D), nq, nk
 
 
 def _items(items) -> np.ndarray:
@@ -129,13 +133,13 @@ class OracleLib:
         lib.oracle_sigmoid.restype = cd
         lib.oracle_sigmoid_grad.argtypes = [cd]
         lib.oracle_sigmoid_grad.restype = cd
-        lib.oracle_fwd_rows.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
+        lib.oracle_fwd_rows.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
                                         i64p, c64, f64p]
-        lib.oracle_dq_rows.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
+        lib.oracle_dq_rows.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
                                        i64p, c64, f64p]
-        lib.oracle_dkdv_rows.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd,
+        lib.oracle_dkdv_rows.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, i32p, i32p, cd,
                                          f64p, i64p, c64, f64p, f64p]
-        lib.oracle_dbias.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
+        lib.oracle_dbias.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, i32p, i32p, cd, f64p,
                                      f64p, f64p]
         lib.oracle_num_threads.restype = ci
         self.lib = lib
@@ -154,11 +158,11 @@ class OracleLib:
 
     def fwd_rows(self, q, k, v, seqlens_q, seqlens_k, alpha, bias, items) -> np.ndarray:
         """O rows for the (z, h, i) triples in ``items``; returns float64 [n, D]."""
-        qa, ka, va, _, dt, (Z, L, H, D), nq, nk = _common(q, k, v, None, seqlens_q, seqlens_k)
+        qa, ka, va, _, dt, (Z, Lq, Lk, H, D), nq, nk = _common(q, k, v, None, seqlens_q, seqlens_k)
         it = _items(items)
         out = np.zeros((it.shape[0], D), dtype=np.float64)
         bz = _bias(bias, Z)
-        self.lib.oracle_fwd_rows(_vp(qa), _vp(ka), _vp(va), dt, Z, L, H, D,
+        self.lib.oracle_fwd_rows(_vp(qa), _vp(ka), _vp(va), dt, Z, Lq, Lk, H, D,
                                  _p(nq, ctypes.c_int32), _p(nk, ctypes.c_int32),
                                  float(alpha), _p(bz, ctypes.c_double), _p(it, ctypes.c_int64),
                                  it.shape[0], _p(out, ctypes.c_double))
@@ -166,11 +170,11 @@ class OracleLib:
 
     def dq_rows(self, q, k, v, dout, seqlens_q, seqlens_k, alpha, bias, items) -> np.ndarray:
         """dQ rows for the (z, h, i) triples in ``items``; float64 [n, D]."""
-        qa, ka, va, da, dt, (Z, L, H, D), nq, nk = _common(q, k, v, dout, seqlens_q, seqlens_k)
+        qa, ka, va, da, dt, (Z, Lq, Lk, H, D), nq, nk = _common(q, k, v, dout, seqlens_q, seqlens_k)
         it = _items(items)
         out = np.zeros((it.shape[0], D), dtype=np.float64)
         bz = _bias(bias, Z)
-        self.lib.oracle_dq_rows(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, L, H, D,
+        self.lib.oracle_dq_rows(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, Lq, Lk, H, D,
                                 _p(nq, ctypes.c_int32), _p(nk, ctypes.c_int32),
                                 float(alpha), _p(bz, ctypes.c_double), _p(it, ctypes.c_int64),
                                 it.shape[0], _p(out, ctypes.c_double))
@@ -178,44 +182,45 @@ class OracleLib:
 
     def dkdv_rows(self, q, k, v, dout, seqlens_q, seqlens_k, alpha, bias, items):
         """(dK rows, dV rows) for the (z, h, j) key triples in ``items``; float64 [n, D] each."""
-        qa, ka, va, da, dt, (Z, L, H, D), nq, nk = _common(q, k, v, dout, seqlens_q, seqlens_k)
+        qa, ka, va, da, dt, (Z, Lq, Lk, H, D), nq, nk = _common(q, k, v, dout, seqlens_q, seqlens_k)
         it = _items(items)
         dk = np.zeros((it.shape[0], D), dtype=np.float64)
         dv = np.zeros((it.shape[0], D), dtype=np.float64)
         bz = _bias(bias, Z)
-        self.lib.oracle_dkdv_rows(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, L, H, D,
+        self.lib.oracle_dkdv_rows(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, Lq, Lk, H, D,
                                   _p(nq, ctypes.c_int32), _p(nk, ctypes.c_int32),
                                   float(alpha), _p(bz, ctypes.c_double), _p(it, ctypes.c_int64),
                                   it.shape[0], _p(dk, ctypes.c_double), _p(dv, ctypes.c_double))
         return dk, dv
 
     def fwd(self, q, k, v, seqlens_q, seqlens_k, alpha, bias) -> np.ndarray:
-        """Full forward O as float64 [Z, L, H, D]."""
-        Z, L, H, D = (int(s) for s in q.shape)
-        rows = self.fwd_rows(q, k, v, seqlens_q, seqlens_k, alpha, bias, all_rows(Z, L, H))
-        return rows.reshape(Z, L, H, D)
+        """Full forward O as float64 [Z, Lq, H, D]."""
+        Z, Lq, H, D = (int(s) for s in q.shape)
+        rows = self.fwd_rows(q, k, v, seqlens_q, seqlens_k, alpha, bias, all_rows(Z, Lq, H))
+        return rows.reshape(Z, Lq, H, D)
 
     def dbias(self, q, k, v, dout, seqlens_q, seqlens_k, alpha, bias) -> np.ndarray:
         """Bias gradient per sample, float64 [Z]: db_z = sum over heads and valid
         (i, j) of dS_ij (paperlayer.ai summary, section 3; gist.science summary,
         section 2.A: x = alpha q.k + b, so dx/db = 1)."""
-        qa, ka, va, da, dt, (Z, L, H, D), nq, nk = _common(q, k, v, dout, seqlens_q, seqlens_k)
+        qa, ka, va, da, dt, (Z, Lq, Lk, H, D), nq, nk = _common(q, k, v, dout, seqlens_q, seqlens_k)
         bz = _bias(bias, Z)
-        rowsum = np.zeros(Z * H * L, dtype=np.float64)
+        rowsum = np.zeros(Z * H * Lq, dtype=np.float64)
         out = np.zeros(Z, dtype=np.float64)
-        self.lib.oracle_dbias(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, L, H, D,
+        self.lib.oracle_dbias(_vp(qa), _vp(ka), _vp(va), _vp(da), dt, Z, Lq, Lk, H, D,
                               _p(nq, ctypes.c_int32), _p(nk, ctypes.c_int32), float(alpha),
                               _p(bz, ctypes.c_double), _p(rowsum, ctypes.c_double),
                               _p(out, ctypes.c_double))
         return out
 
     def bwd(self, q, k, v, dout, seqlens_q, seqlens_k, alpha, bias):
-        """Full backward (dQ, dK, dV) as float64 [Z, L, H, D] each."""
-        Z, L, H, D = (int(s) for s in q.shape)
-        rows = all_rows(Z, L, H)
-        dq = self.dq_rows(q, k, v, dout, seqlens_q, seqlens_k, alpha, bias, rows)
-        dk, dv = self.dkdv_rows(q, k, v, dout, seqlens_q, seqlens_k, alpha, bias, rows)
-        return (dq.reshape(Z, L, H, D), dk.reshape(Z, L, H, D), dv.reshape(Z, L, H, D))
+        """Full backward: dQ as float64 [Z, Lq, H, D], dK and dV as [Z, Lk, H, D]."""
+        Z, Lq, H, D = (int(s) for s in q.shape)
+        Lk = int(k.shape[1])
+        dq = self.dq_rows(q, k, v, dout, seqlens_q, seqlens_k, alpha, bias, all_rows(Z, Lq, H))
+        dk, dv = self.dkdv_rows(q, k, v, dout, seqlens_q, seqlens_k, alpha, bias,
+                                all_rows(Z, Lk, H))
+        return (dq.reshape(Z, Lq, H, D), dk.reshape(Z, Lk, H, D), dv.reshape(Z, Lk, H, D))
 
 
 def default() -> OracleLib:

@@ -32,7 +32,10 @@
  *     kernel pages describe (the approximation is what the oracle judges).
  *
  * Layout of every tensor: [Z][L][H][D], contiguous; element (z,l,h,d) sits at
- * ((z*L + l)*H + h)*D + d.  dtype 0 = bf16 (raw uint16 bits), 1 = fp32.
+ * ((z*L + l)*H + h)*D + d, with L = Lq for Q, dO and the query-side outputs
+ * (O, dQ) and L = Lk for K, V, dK, dV (Lq = Lk for self-attention; a shorter
+ * query slice against all keys is the context-parallel case).
+ * dtype 0 = bf16 (raw uint16 bits), 1 = fp32.
  * Row lists are int64 triples (z, h, row).  Outputs are double, D per row.
  * bias_z holds one bias per sample (double[Z]).
  *
@@ -73,18 +76,21 @@ double oracle_sigmoid_grad(double x) {
     return p * (1.0 - p);
 }
 
-/* score x_ij = alpha * sum_d Q[i,d] K[j,d] + b for one (z, h) */
+/* score x_ij = alpha * sum_d Q[i,d] K[j,d] + b for one (z, h); Q and dO rows are
+ * laid out with the query length Lq, K and V rows with the key length Lk */
 static double score(const void *q, const void *k, int dtype, int64_t z, int64_t h,
-                    int64_t i, int64_t j, int L, int H, int D, double alpha, double bias) {
-    int64_t qo = offset_of(z, i, h, L, H, D), ko = offset_of(z, j, h, L, H, D);
+                    int64_t i, int64_t j, int Lq, int Lk, int H, int D, double alpha,
+                    double bias) {
+    int64_t qo = offset_of(z, i, h, Lq, H, D), ko = offset_of(z, j, h, Lk, H, D);
     double s = 0.0;
     for (int d = 0; d < D; ++d) s += load_elem(q, dtype, qo + d) * load_elem(k, dtype, ko + d);
     return alpha * s + bias;
 }
 
+/* sum_d A[i,d] B[j,d] with A in the query layout (Lq) and B in the key layout (Lk) */
 static double dot_rows(const void *a, const void *b, int dtype, int64_t z, int64_t h,
-                       int64_t i, int64_t j, int L, int H, int D) {
-    int64_t ao = offset_of(z, i, h, L, H, D), bo = offset_of(z, j, h, L, H, D);
+                       int64_t i, int64_t j, int Lq, int Lk, int H, int D) {
+    int64_t ao = offset_of(z, i, h, Lq, H, D), bo = offset_of(z, j, h, Lk, H, D);
     double s = 0.0;
     for (int d = 0; d < D; ++d) s += load_elem(a, dtype, ao + d) * load_elem(b, dtype, bo + d);
     return s;
@@ -94,7 +100,7 @@ static int clamp_len(int n, int L) { return n < 0 ? 0 : (n > L ? L : n); }
 
 /* Forward rows: O[z, i, h, :] = [i < n_q] sum_{j < n_k} sigma(x_ij) V[z, j, h, :]. */
 void oracle_fwd_rows(const void *q, const void *k, const void *v, int dtype,
-                     int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
+                     int Z, int Lq, int Lk, int H, int D, const int32_t *nq, const int32_t *nk,
                      double alpha, const double *bias_z, const int64_t *items, int64_t nitems,
                      double *out) {
     (void)Z;
@@ -103,12 +109,12 @@ void oracle_fwd_rows(const void *q, const void *k, const void *v, int dtype,
         int64_t z = items[3 * t], h = items[3 * t + 1], i = items[3 * t + 2];
         double *o = out + t * D;
         for (int d = 0; d < D; ++d) o[d] = 0.0;
-        int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        int n_q = clamp_len(nq[z], Lq), n_k = clamp_len(nk[z], Lk);
         const double bias = bias_z[z];
         if (i >= n_q) continue;
         for (int64_t j = 0; j < n_k; ++j) {
-            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
-            int64_t vo = offset_of(z, j, h, L, H, D);
+            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, Lq, Lk, H, D, alpha, bias));
+            int64_t vo = offset_of(z, j, h, Lk, H, D);
             for (int d = 0; d < D; ++d) o[d] += p * load_elem(v, dtype, vo + d);
         }
     }
@@ -117,7 +123,7 @@ void oracle_fwd_rows(const void *q, const void *k, const void *v, int dtype,
 /* dQ rows: dQ[z, i, h, :] = [i < n_q] alpha sum_{j < n_k} dS_ij K[z, j, h, :],
  * dS_ij = P_ij (1 - P_ij) (dO_i . V_j). */
 void oracle_dq_rows(const void *q, const void *k, const void *v, const void *dout, int dtype,
-                    int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
+                    int Z, int Lq, int Lk, int H, int D, const int32_t *nq, const int32_t *nk,
                     double alpha, const double *bias_z, const int64_t *items, int64_t nitems,
                     double *out) {
     (void)Z;
@@ -126,14 +132,14 @@ void oracle_dq_rows(const void *q, const void *k, const void *v, const void *dou
         int64_t z = items[3 * t], h = items[3 * t + 1], i = items[3 * t + 2];
         double *g = out + t * D;
         for (int d = 0; d < D; ++d) g[d] = 0.0;
-        int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        int n_q = clamp_len(nq[z], Lq), n_k = clamp_len(nk[z], Lk);
         const double bias = bias_z[z];
         if (i >= n_q) continue;
         for (int64_t j = 0; j < n_k; ++j) {
-            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
-            double dp = dot_rows(dout, v, dtype, z, h, i, j, L, H, D);
+            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, Lq, Lk, H, D, alpha, bias));
+            double dp = dot_rows(dout, v, dtype, z, h, i, j, Lq, Lk, H, D);
             double ds = p * (1.0 - p) * dp;
-            int64_t ko = offset_of(z, j, h, L, H, D);
+            int64_t ko = offset_of(z, j, h, Lk, H, D);
             for (int d = 0; d < D; ++d) g[d] += ds * load_elem(k, dtype, ko + d);
         }
         for (int d = 0; d < D; ++d) g[d] *= alpha;
@@ -144,7 +150,7 @@ void oracle_dq_rows(const void *q, const void *k, const void *v, const void *dou
  *   dV[z, j, h, :] = [j < n_k] sum_{i < n_q} P_ij dO[z, i, h, :]
  *   dK[z, j, h, :] = [j < n_k] alpha sum_{i < n_q} dS_ij Q[z, i, h, :] */
 void oracle_dkdv_rows(const void *q, const void *k, const void *v, const void *dout, int dtype,
-                      int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
+                      int Z, int Lq, int Lk, int H, int D, const int32_t *nq, const int32_t *nk,
                       double alpha, const double *bias_z, const int64_t *items, int64_t nitems,
                       double *dk_out, double *dv_out) {
     (void)Z;
@@ -153,14 +159,14 @@ void oracle_dkdv_rows(const void *q, const void *k, const void *v, const void *d
         int64_t z = items[3 * t], h = items[3 * t + 1], j = items[3 * t + 2];
         double *gk = dk_out + t * D, *gv = dv_out + t * D;
         for (int d = 0; d < D; ++d) { gk[d] = 0.0; gv[d] = 0.0; }
-        int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        int n_q = clamp_len(nq[z], Lq), n_k = clamp_len(nk[z], Lk);
         const double bias = bias_z[z];
         if (j >= n_k) continue;
         for (int64_t i = 0; i < n_q; ++i) {
-            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
-            double dp = dot_rows(dout, v, dtype, z, h, i, j, L, H, D);
+            double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, Lq, Lk, H, D, alpha, bias));
+            double dp = dot_rows(dout, v, dtype, z, h, i, j, Lq, Lk, H, D);
             double ds = p * (1.0 - p) * dp;
-            int64_t qo = offset_of(z, i, h, L, H, D);
+            int64_t qo = offset_of(z, i, h, Lq, H, D);
             for (int d = 0; d < D; ++d) {
                 gv[d] += p * load_elem(dout, dtype, qo + d);
                 gk[d] += ds * load_elem(q, dtype, qo + d);
@@ -175,19 +181,19 @@ void oracle_dkdv_rows(const void *q, const void *k, const void *v, const void *d
  * in ascending j; the partials are then added in ascending (h, i) order per
  * sample, so the result does not depend on the thread count. */
 void oracle_dbias(const void *q, const void *k, const void *v, const void *dout, int dtype,
-                  int Z, int L, int H, int D, const int32_t *nq, const int32_t *nk,
+                  int Z, int Lq, int Lk, int H, int D, const int32_t *nq, const int32_t *nk,
                   double alpha, const double *bias_z, double *rowsum, double *dbias) {
-    const int64_t nrows = (int64_t)Z * H * L;
+    const int64_t nrows = (int64_t)Z * H * Lq;
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t t = 0; t < nrows; ++t) {
-        int64_t z = t / ((int64_t)H * L), h = (t / L) % H, i = t % L;
+        int64_t z = t / ((int64_t)H * Lq), h = (t / Lq) % H, i = t % Lq;
         double acc = 0.0;
-        int n_q = clamp_len(nq[z], L), n_k = clamp_len(nk[z], L);
+        int n_q = clamp_len(nq[z], Lq), n_k = clamp_len(nk[z], Lk);
         const double bias = bias_z[z];
         if (i < n_q) {
             for (int64_t j = 0; j < n_k; ++j) {
-                double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));
-                double dp = dot_rows(dout, v, dtype, z, h, i, j, L, H, D);
+                double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, Lq, Lk, H, D, alpha, bias));
+                double dp = dot_rows(dout, v, dtype, z, h, i, j, Lq, Lk, H, D);
                 acc += p * (1.0 - p) * dp;
             }
         }
@@ -195,7 +201,7 @@ void oracle_dbias(const void *q, const void *k, const void *v, const void *dout,
     }
     for (int64_t z = 0; z < Z; ++z) {
         double s = 0.0;
-        for (int64_t r = 0; r < (int64_t)H * L; ++r) s += rowsum[z * H * L + r];
+        for (int64_t r = 0; r < (int64_t)H * Lq; ++r) s += rowsum[z * H * Lq + r];
         dbias[z] = s;
     }
 }

@@ -16,7 +16,9 @@ mathematics fix:
 * central finite differences of the oracle's own (pinned) forward;
 * a per-sample bias (paperlayer.ai summary, section 3: b = -log(n)) and its
   gradient db against torch autograd, the alpha = 0 closed form and a finite
-  difference.
+  difference;
+* rectangular problems (a query slice against all keys, Lq != Lk) against
+  torch autograd and against the square problem they embed in.
 
 ``tests/test_oracle_pins.py`` runs them on the real oracle and
 ``tests/test_oracle_mutants.py`` shows that builds with one plausible mistake
@@ -413,6 +415,63 @@ def pin_dbias_finite_difference(orc):
             raise AssertionError(f"db[{z}]: oracle {db[z]} vs finite difference {fd}")
 
 
+# ---------------------------------------------------------------- rectangular (Lq != Lk)
+
+
+def _rect_case(seed, Z=2, Lq=4, Lk=7, H=2, D=3, nq=(4, 2), nk=(7, 5), scale=1.0):
+    q = _rand((Z, Lq, H, D), seed, scale)
+    k = _rand((Z, Lk, H, D), seed + 1, scale)
+    v = _rand((Z, Lk, H, D), seed + 2)
+    do = _rand((Z, Lq, H, D), seed + 3)
+    return q, k, v, do, np.asarray(nq, np.int32), np.asarray(nk, np.int32)
+
+
+def pin_rectangular_autograd(orc):
+    """A query slice of length Lq against Lk keys (the context-parallel shape)
+    against torch fp64 autograd with the same masks."""
+    for seed, kw in [(220, {}), (230, dict(Z=1, Lq=6, Lk=3, H=3, D=4, nq=(5,), nk=(3,))),
+                     (240, dict(Z=3, Lq=2, Lk=9, H=1, D=2, nq=(2, 0, 1), nk=(9, 4, 0)))]:
+        q, k, v, do, nq, nk = _rect_case(seed, **kw)
+        Z, Lq, H, D = q.shape
+        Lk = k.shape[1]
+        alpha, bias = 0.52, -0.9
+        tq, tk, tv = (torch.tensor(a.astype(np.float64), requires_grad=True) for a in (q, k, v))
+        tdo = torch.from_numpy(do.astype(np.float64))
+        kmask = torch.zeros((Z, Lk), dtype=torch.float64)
+        qmask = torch.zeros((Z, Lq), dtype=torch.float64)
+        for z in range(Z):
+            kmask[z, : nk[z]] = 1.0
+            qmask[z, : nq[z]] = 1.0
+        sc = alpha * torch.einsum("zihd,zjhd->zhij", tq, tk) + bias
+        pr = torch.sigmoid(sc) * kmask[:, None, None, :]
+        o = torch.einsum("zhij,zjhd->zihd", pr, tv) * qmask[:, :, None, None]
+        (o * tdo).sum().backward()
+        _close(orc.fwd(q, k, v, nq, nk, alpha, bias), o.detach().numpy(), 1e-12, 1e-13,
+               f"rectangular forward vs torch (seed {seed})")
+        dq, dk, dv = orc.bwd(q, k, v, do, nq, nk, alpha, bias)
+        _close(dq, tq.grad.numpy(), 1e-11, 1e-12, f"rectangular dQ (seed {seed})")
+        _close(dk, tk.grad.numpy(), 1e-11, 1e-12, f"rectangular dK (seed {seed})")
+        _close(dv, tv.grad.numpy(), 1e-11, 1e-12, f"rectangular dV (seed {seed})")
+
+
+def pin_rectangular_embedding(orc):
+    """A rectangular problem equals the square one whose Q and dO are padded with
+    extra rows beyond n_q (they are padding, so they change nothing)."""
+    q, k, v, do, nq, nk = _rect_case(250, Z=2, Lq=3, Lk=6, H=2, D=3, nq=(3, 2), nk=(6, 4))
+    alpha, bias = 0.7, -0.4
+    Lq, Lk = q.shape[1], k.shape[1]
+    pad = lambda a: np.concatenate([a, _rand((2, Lk - Lq) + a.shape[2:], 260)], axis=1)
+    qs, dos = pad(q), pad(do)
+    o_r = orc.fwd(q, k, v, nq, nk, alpha, bias)
+    o_s = orc.fwd(qs, k, v, nq, nk, alpha, bias)
+    _close(o_r, o_s[:, :Lq], 0, 0, "rectangular O = square O rows")
+    g_r = orc.bwd(q, k, v, do, nq, nk, alpha, bias)
+    g_s = orc.bwd(qs, k, v, dos, nq, nk, alpha, bias)
+    _close(g_r[0], g_s[0][:, :Lq], 0, 0, "rectangular dQ = square dQ rows")
+    _close(g_r[1], g_s[1], 0, 0, "rectangular dK = square dK")
+    _close(g_r[2], g_s[2], 0, 0, "rectangular dV = square dV")
+
+
 ALL_PINS = [
     pin_sigmoid_closed_forms,
     pin_sigmoid_derivative,
@@ -431,4 +490,6 @@ ALL_PINS = [
     pin_per_sample_bias_slices,
     pin_dbias_alpha_zero,
     pin_dbias_finite_difference,
+    pin_rectangular_autograd,
+    pin_rectangular_embedding,
 ]

@@ -19,8 +19,8 @@ MUTANTS = [
     ("sigmoid-sign", "return 1.0 / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(x));", None),
     ("sigmoid-grad-dropped-term", "return p * (1.0 - p);", "return p;", None),
     ("fwd-no-query-mask", "if (i >= n_q) continue;", "", 0),
-    ("fwd-no-key-mask", "for (int64_t j = 0; j < n_k; ++j) {", "for (int64_t j = 0; j < L; ++j) {", 0),
-    ("dq-no-key-mask", "for (int64_t j = 0; j < n_k; ++j) {", "for (int64_t j = 0; j < L; ++j) {", 1),
+    ("fwd-no-key-mask", "for (int64_t j = 0; j < n_k; ++j) {", "for (int64_t j = 0; j < Lk; ++j) {", 0),
+    ("dq-no-key-mask", "for (int64_t j = 0; j < n_k; ++j) {", "for (int64_t j = 0; j < Lk; ++j) {", 1),
     ("dq-dropped-sigma-prime", "double ds = p * (1.0 - p) * dp;", "double ds = p * dp;", 0),
     ("dkdv-dropped-sigma-prime", "double ds = p * (1.0 - p) * dp;", "double ds = p * dp;", 1),
     ("dq-dropped-alpha", "for (int d = 0; d < D; ++d) g[d] *= alpha;", "", None),
@@ -29,17 +29,20 @@ MUTANTS = [
      "gv[d] += p * load_elem(q, dtype, qo + d);", None),
     ("dk-wrong-operand", "gk[d] += ds * load_elem(q, dtype, qo + d);",
      "gk[d] += ds * load_elem(k, dtype, qo + d);", None),
-    ("dkdv-transposed-score", "double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, L, H, D, alpha, bias));",
-     "double p = oracle_sigmoid(score(q, k, dtype, z, h, j, i, L, H, D, alpha, bias));", 2),
-    ("dq-dp-wrong-operand", "double dp = dot_rows(dout, v, dtype, z, h, i, j, L, H, D);",
-     "double dp = dot_rows(dout, k, dtype, z, h, i, j, L, H, D);", 0),
-    ("dkdv-padded-queries-flow", "for (int64_t i = 0; i < n_q; ++i) {", "for (int64_t i = 0; i < L; ++i) {", None),
+    ("dkdv-transposed-score",
+     "double p = oracle_sigmoid(score(q, k, dtype, z, h, i, j, Lq, Lk, H, D, alpha, bias));",
+     "double p = oracle_sigmoid(score(q, k, dtype, z, h, j, i, Lq, Lk, H, D, alpha, bias));", 2),
+    ("dq-dp-wrong-operand", "double dp = dot_rows(dout, v, dtype, z, h, i, j, Lq, Lk, H, D);",
+     "double dp = dot_rows(dout, k, dtype, z, h, i, j, Lq, Lk, H, D);", 0),
+    ("dkdv-padded-queries-flow", "for (int64_t i = 0; i < n_q; ++i) {", "for (int64_t i = 0; i < Lq; ++i) {", None),
+    ("key-rows-in-query-layout", "int64_t ko = offset_of(z, j, h, Lk, H, D);",
+     "int64_t ko = offset_of(z, j, h, Lq, H, D);", None),
     ("dkdv-no-key-row-mask", "if (j >= n_k) continue;", "", None),
     ("layout-h-l-swapped", "return ((z * L + l) * H + h) * (int64_t)D;",
      "return ((z * H + h) * L + l) * (int64_t)D;", None),
     ("dbias-dropped-sigma-prime", "acc += p * (1.0 - p) * dp;", "acc += p * dp;", None),
-    ("dbias-no-key-mask", "for (int64_t j = 0; j < n_k; ++j) {", "for (int64_t j = 0; j < L; ++j) {", 2),
-    ("dbias-no-query-mask", "if (i < n_q) {", "if (i < L) {", None),
+    ("dbias-no-key-mask", "for (int64_t j = 0; j < n_k; ++j) {", "for (int64_t j = 0; j < Lk; ++j) {", 2),
+    ("dbias-no-query-mask", "if (i < n_q) {", "if (i < Lq) {", None),
     ("bias-per-sample-wrong-index", "const double bias = bias_z[z];", "const double bias = bias_z[0];", None),
     ("bf16-widening", "uint32_t bits = ((uint32_t)b) << 16;", "uint32_t bits = ((uint32_t)b) << 15;", None),
     ("fwd-value-from-key", "for (int d = 0; d < D; ++d) o[d] += p * load_elem(v, dtype, vo + d);",
