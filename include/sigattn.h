@@ -118,6 +118,25 @@ sigattn_status sigattn_bwd_dkdv(const void *q, const void *k, const void *v, con
                                 const int32_t *seqlens_k, int Z, int L, int H, int D,
                                 float alpha, float bias, sigattn_dtype dtype, void *stream);
 
+/* Queries and keys of different padded lengths: q, dout, o, dq are
+ * [Z][Lq][H][D]; k, v, dk, dv are [Z][Lk][H][D]; n_q <= Lq and n_k <= Lk.
+ * This is the shape of one rank's work when a sequence is split across GPUs
+ * (context parallelism): its slice of queries against every key, and dK, dV
+ * contributions of its queries to every key, which the ranks then add up.
+ * Since sigma needs no row normalisation, those contributions are plain sums
+ * (the operation as in sigattn_fwd / sigattn_bwd, gist.science summary,
+ * section 2.A).  Lq = Lk gives exactly sigattn_fwd / sigattn_bwd.
+ * Errors as sigattn_fwd / sigattn_bwd, plus SIGATTN_ERR_INVALID_ARG when
+ * exactly one of Lq, Lk is zero (both zero, or Z or H zero: nothing to do). */
+sigattn_status sigattn_fwd_rect(const void *q, const void *k, const void *v, void *o,
+                                const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int Lq,
+                                int Lk, int H, int D, float alpha, float bias, sigattn_dtype dtype,
+                                void *stream);
+sigattn_status sigattn_bwd_rect(const void *q, const void *k, const void *v, const void *dout,
+                                void *dq, void *dk, void *dv, const int32_t *seqlens_q,
+                                const int32_t *seqlens_k, int Z, int Lq, int Lk, int H, int D,
+                                float alpha, float bias, sigattn_dtype dtype, void *stream);
+
 /* Per-sample bias and its gradient.
  *
  * The pages set the bias to b = -log(n) (paperlayer.ai summary, section 3,

@@ -22,7 +22,7 @@ __all__ = [
     "last_device_status", "set_wait_timeout_ns", "selftest_wait_timeout", "status_string",
     "version", "library_path", "load_library", "SIGMOID_TANH", "SIGMOID_EXP", "EXPORTS",
     "SigmoidAttention", "bwd_dq", "bwd_dkdv", "last_cuda_error", "fwd_noalloc", "NOALLOC_MAX_Z",
-    "fwd_bias", "bwd_bias", "dbias_workspace_bytes",
+    "fwd_bias", "bwd_bias", "dbias_workspace_bytes", "fwd_rect", "bwd_rect",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -50,6 +50,7 @@ EXPORTS = (
     "sigattn_last_device_status", "sigattn_set_wait_timeout_ns", "sigattn_selftest_wait_timeout",
     "sigattn_last_cuda_error", "sigattn_status_string", "sigattn_version",
     "sigattn_fwd_noalloc", "sigattn_fwd_bias", "sigattn_bwd_bias", "sigattn_dbias_workspace_bytes",
+    "sigattn_fwd_rect", "sigattn_bwd_rect",
 )
 
 
@@ -86,6 +87,11 @@ def load_library():
         lib.sigattn_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf,
                                          ci, vp]
         lib.sigattn_bwd_dkdv.restype = ci
+        lib.sigattn_fwd_rect.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, cf, ci, vp]
+        lib.sigattn_fwd_rect.restype = ci
+        lib.sigattn_bwd_rect.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf,
+                                         cf, ci, vp]
+        lib.sigattn_bwd_rect.restype = ci
         lib.sigattn_fwd_bias.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, vp, ci, vp]
         lib.sigattn_fwd_bias.restype = ci
         lib.sigattn_bwd_bias.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf,
@@ -213,6 +219,49 @@ def bwd_dkdv(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, dk=
         seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, L, H, D, float(alpha), float(bias),
         _dtype_code(q), _stream_ptr(q)), "sigattn_bwd_dkdv")
     return dk, dv
+
+
+def _check_rect(queries, keys, seqlens):
+    """Shapes of the rectangular calls: query-side tensors [Z, Lq, H, D] share one
+    shape, key-side tensors [Z, Lk, H, D] another, with the same Z, H, D, dtype
+    and device."""
+    _check_inputs(queries, seqlens)
+    _check_inputs(keys, [])
+    a, b = queries[0], keys[0]
+    if a.shape[0] != b.shape[0] or a.shape[2:] != b.shape[2:] or a.dtype != b.dtype \
+            or a.device != b.device:
+        raise ValueError("queries and keys must share Z, H, D, dtype and device")
+
+
+def fwd_rect(q, k, v, seqlens_q, seqlens_k, alpha: float, bias: float, out=None):
+    """Forward with q [Z, Lq, H, D] against k, v [Z, Lk, H, D]; O is [Z, Lq, H, D]."""
+    import torch
+    out = torch.empty_like(q) if out is None else out
+    _check_rect([q, out], [k, v], [seqlens_q, seqlens_k])
+    Z, Lq, H, D = (int(x) for x in q.shape)
+    Lk = int(k.shape[1])
+    _check(load_library().sigattn_fwd_rect(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), seqlens_q.data_ptr(),
+        seqlens_k.data_ptr(), Z, Lq, Lk, H, D, float(alpha), float(bias), _dtype_code(q),
+        _stream_ptr(q)), "sigattn_fwd_rect")
+    return out
+
+
+def bwd_rect(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, dq=None, dk=None,
+             dv=None):
+    """Backward of ``fwd_rect``: dQ [Z, Lq, H, D]; dK, dV [Z, Lk, H, D]."""
+    import torch
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_rect([q, dout, dq], [k, v, dk, dv], [seqlens_q, seqlens_k])
+    Z, Lq, H, D = (int(x) for x in q.shape)
+    Lk = int(k.shape[1])
+    _check(load_library().sigattn_bwd_rect(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+        dv.data_ptr(), seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, Lq, Lk, H, D, float(alpha),
+        float(bias), _dtype_code(q), _stream_ptr(q)), "sigattn_bwd_rect")
+    return dq, dk, dv
 
 
 def _check_bias(bias, ref):

@@ -33,7 +33,7 @@ struct BwdParams {
     __nv_bfloat16 *dv;
     const int *seqlens_q;
     const int *seqlens_k;
-    int L, H;
+    int Lq, Lk, H;          // padded lengths of Q, dO, dQ and of K, V, dK, dV; heads
     float alpha, bias;
     int *status;
     uint64_t timeout_ns;
@@ -178,12 +178,12 @@ __global__ void __launch_bounds__(384, 1)
 
     const int warp = warp_id(), lane = lane_id();
     const int z = blockIdx.z, h = blockIdx.y, qtile = blockIdx.x;
-    const int L = p.L;
+    const int L = p.Lq;     // rows of this kernel's tiles and outputs: queries
     int nq = p.seqlens_q[z], nk = p.seqlens_k[z];
-    if (nq < 0 || nq > L || nk < 0 || nk > L) {
+    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
         if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
         nq = min(max(nq, 0), L);
-        nk = min(max(nk, 0), L);
+        nk = min(max(nk, 0), p.Lk);
     }
     const int nkv = (nk + 127) / 128;
     const bool work = qtile * 128 < nq && nkv > 0;
@@ -458,11 +458,11 @@ __global__ void __launch_bounds__(384, 1)
 
     const int warp = warp_id(), lane = lane_id();
     const int z = blockIdx.z, h = blockIdx.y, ktile = blockIdx.x;
-    const int L = p.L;
+    const int L = p.Lk;     // rows of this kernel's tiles and outputs: keys
     int nq = p.seqlens_q[z], nk = p.seqlens_k[z];
-    if (nq < 0 || nq > L || nk < 0 || nk > L) {
+    if (nq < 0 || nq > p.Lq || nk < 0 || nk > L) {
         if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
-        nq = min(max(nq, 0), L);
+        nq = min(max(nq, 0), p.Lq);
         nk = min(max(nk, 0), L);
     }
     const int nqt = (nq + 127) / 128;

@@ -30,7 +30,7 @@ struct F32Params {
     const float *q, *k, *v, *dout;
     float *o, *dq, *dk, *dv;
     const int *seqlens_q, *seqlens_k;
-    int Z, L, H;
+    int Z, Lq, Lk, H;       // batch, padded lengths of Q / dO / O / dQ and of K / V / dK / dV
     float alpha, bias;
     int *status;
     const float *bias_z;   // device float[Z], one bias per sample; null: the scalar `bias`
@@ -40,24 +40,25 @@ struct F32Params {
 __device__ __forceinline__ void clamp_lengths(const F32Params &p, int z, int &nq, int &nk) {
     nq = p.seqlens_q[z];
     nk = p.seqlens_k[z];
-    if (nq < 0 || nq > p.L || nk < 0 || nk > p.L) {
+    if (nq < 0 || nq > p.Lq || nk < 0 || nk > p.Lk) {
         if ((threadIdx.x & 31) == 0) record_status(p.status, kStatusSeqlenRange);
-        nq = min(max(nq, 0), p.L);
-        nk = min(max(nk, 0), p.L);
+        nq = min(max(nq, 0), p.Lq);
+        nk = min(max(nk, 0), p.Lk);
     }
 }
 
-// rows are enumerated in [Z][L][H] order, so row r starts at r * D
+// rows are enumerated in [Z][L][H] order (L = Lq for query rows, Lk for key
+// rows), so row r starts at r * D
 template <int D>
 __global__ void __launch_bounds__(256) f32_fwd_kernel(const F32Params p) {
     constexpr int E = D / 32;
     const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    const int64_t rows = static_cast<int64_t>(p.Z) * p.L * p.H;
+    const int64_t rows = static_cast<int64_t>(p.Z) * p.Lq * p.H;
     if (r >= rows) return;
     const int h = static_cast<int>(r % p.H);
-    const int i = static_cast<int>((r / p.H) % p.L);
-    const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.L));
+    const int i = static_cast<int>((r / p.H) % p.Lq);
+    const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.Lq));
     int nq, nk;
     clamp_lengths(p, z, nq, nk);
     const float bias = bias_of(p.bias_z, p.bias, z);
@@ -69,7 +70,7 @@ __global__ void __launch_bounds__(256) f32_fwd_kernel(const F32Params p) {
 #pragma unroll
         for (int e = 0; e < E; ++e) qv[e] = p.q[r * D + lane + 32 * e];
         for (int j = 0; j < nk; ++j) {
-            const int64_t kr = (static_cast<int64_t>(z) * p.L + j) * p.H + h;
+            const int64_t kr = (static_cast<int64_t>(z) * p.Lk + j) * p.H + h;
             float s = 0.0f;
 #pragma unroll
             for (int e = 0; e < E; ++e) s = fmaf(qv[e], p.k[kr * D + lane + 32 * e], s);
@@ -89,11 +90,11 @@ __global__ void __launch_bounds__(256) f32_dq_kernel(const F32Params p) {
     constexpr int E = D / 32;
     const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    const int64_t rows = static_cast<int64_t>(p.Z) * p.L * p.H;
+    const int64_t rows = static_cast<int64_t>(p.Z) * p.Lq * p.H;
     if (r >= rows) return;
     const int h = static_cast<int>(r % p.H);
-    const int i = static_cast<int>((r / p.H) % p.L);
-    const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.L));
+    const int i = static_cast<int>((r / p.H) % p.Lq);
+    const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.Lq));
     int nq, nk;
     clamp_lengths(p, z, nq, nk);
     const float bias = bias_of(p.bias_z, p.bias, z);
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(256) f32_dq_kernel(const F32Params p) {
             gv[e] = p.dout[r * D + lane + 32 * e];
         }
         for (int j = 0; j < nk; ++j) {
-            const int64_t kr = (static_cast<int64_t>(z) * p.L + j) * p.H + h;
+            const int64_t kr = (static_cast<int64_t>(z) * p.Lk + j) * p.H + h;
             float s = 0.0f, dp = 0.0f;
 #pragma unroll
             for (int e = 0; e < E; ++e) {
@@ -136,11 +137,11 @@ __global__ void __launch_bounds__(256) f32_dkdv_kernel(const F32Params p) {
     constexpr int E = D / 32;
     const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    const int64_t rows = static_cast<int64_t>(p.Z) * p.L * p.H;
+    const int64_t rows = static_cast<int64_t>(p.Z) * p.Lk * p.H;
     if (r >= rows) return;
     const int h = static_cast<int>(r % p.H);
-    const int j = static_cast<int>((r / p.H) % p.L);
-    const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.L));
+    const int j = static_cast<int>((r / p.H) % p.Lk);
+    const int z = static_cast<int>(r / (static_cast<int64_t>(p.H) * p.Lk));
     int nq, nk;
     clamp_lengths(p, z, nq, nk);
     const float bias = bias_of(p.bias_z, p.bias, z);
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(256) f32_dkdv_kernel(const F32Params p) {
             vv[e] = p.v[r * D + lane + 32 * e];
         }
         for (int i = 0; i < nq; ++i) {
-            const int64_t qr = (static_cast<int64_t>(z) * p.L + i) * p.H + h;
+            const int64_t qr = (static_cast<int64_t>(z) * p.Lq + i) * p.H + h;
             float s = 0.0f, dp = 0.0f;
 #pragma unroll
             for (int e = 0; e < E; ++e) {

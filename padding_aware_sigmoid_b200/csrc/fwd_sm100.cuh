@@ -37,7 +37,7 @@ struct FwdParams {
     __nv_bfloat16 *o;
     const int *seqlens_q;
     const int *seqlens_k;
-    int L, H;
+    int Lq, Lk, H;          // padded lengths of Q (and O) and of K, V; heads
     float alpha, bias;
     int *status;
     uint64_t timeout_ns;
@@ -109,13 +109,13 @@ __global__ void __launch_bounds__(384, 1)
     const int warp = warp_id(), lane = lane_id();
     const int z = blockIdx.z, h = blockIdx.y;
     const int qtile0 = blockIdx.x * 2;
-    const int L = p.L;
+    const int L = p.Lq;     // query rows of this problem (O has the same layout)
 
     int nq = p.seqlens_q[z], nk = p.seqlens_k[z];
-    if (nq < 0 || nq > L || nk < 0 || nk > L) {
+    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
         if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
         nq = min(max(nq, 0), L);
-        nk = min(max(nk, 0), L);
+        nk = min(max(nk, 0), p.Lk);
     }
     const int ntiles = (qtile0 * Lay::BM < nq ? 1 : 0) + ((qtile0 + 1) * Lay::BM < nq ? 1 : 0);
     const int nkv = (nk + Lay::BN - 1) / Lay::BN;

@@ -110,6 +110,23 @@ sigattn_status check_shape(int Z, int L, int H, int D, sigattn_dtype dtype, bool
     return SIGATTN_OK;
 }
 
+// check_shape for queries and keys of padded lengths Lq and Lk: both zero is an
+// empty problem, exactly one zero is an error (the other side's outputs would
+// have rows but no keys or queries to read).
+sigattn_status check_lengths(int Z, int Lq, int Lk, int H, int D, sigattn_dtype dtype,
+                             bool *empty) {
+    bool eq = false, ek = false;
+    sigattn_status s = check_shape(Z, Lq, H, D, dtype, &eq);
+    if (s != SIGATTN_OK) return s;
+    if ((s = check_shape(Z, Lk, H, D, dtype, &ek)) != SIGATTN_OK) return s;
+    if (Z == 0 || H == 0 || (Lq == 0 && Lk == 0)) {
+        *empty = true;
+        return SIGATTN_OK;
+    }
+    *empty = false;
+    return (Lq == 0 || Lk == 0) ? SIGATTN_ERR_INVALID_ARG : SIGATTN_OK;
+}
+
 template <typename... KArgs, typename... Args>
 sigattn_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                       cudaStream_t stream, Args... args) {
@@ -141,9 +158,10 @@ enum BwdParts : int { kPartDq = 1, kPartDkdv = 2 };
 
 template <int D, int MODE>
 sigattn_status bwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                        const CUtensorMap &mdo, const BwdParams &p, int Z, int L, int H,
-                        int parts, cudaStream_t st) {
-    dim3 grid((L + 127) / 128, H, Z);
+                        const CUtensorMap &mdo, const BwdParams &p, int Z, int Lq, int Lk,
+                        int H, int parts, cudaStream_t st) {
+    dim3 grid((Lq + 127) / 128, H, Z);      // dQ: one CTA per query tile
+    dim3 grid_kv((Lk + 127) / 128, H, Z);   // dK/dV: one CTA per key tile
     constexpr int SX = BwdStages<D>::X, SY = BwdStages<D>::Y;
     constexpr size_t smem = BwdLayout<D, SX, SY>::SMEM_ALLOC;
     if (parts & kPartDq) {
@@ -156,7 +174,7 @@ sigattn_status bwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
         if (s != SIGATTN_OK) return s;
     }
     if (parts & kPartDkdv)
-        return launch(bwd_dkdv_kernel<D, MODE, SX, SY>, grid, dim3(384), smem, st, mq, mk, mv,
+        return launch(bwd_dkdv_kernel<D, MODE, SX, SY>, grid_kv, dim3(384), smem, st, mq, mk, mv,
                       mdo, p);
     return SIGATTN_OK;
 }
@@ -172,11 +190,11 @@ int64_t dbias_partials_per_sample(int L, int H, sigattn_dtype dtype) {
 // float[Z]) receives the bias gradient when not null, through `work`.
 sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void *dout, void *dq,
                         void *dk, void *dv, const int32_t *seqlens_q, const int32_t *seqlens_k,
-                        int Z, int L, int H, int D, float alpha, float bias, sigattn_dtype dtype,
-                        void *stream, int parts, const float *bias_z = nullptr,
+                        int Z, int Lq, int Lk, int H, int D, float alpha, float bias,
+                        sigattn_dtype dtype, void *stream, int parts, const float *bias_z = nullptr,
                         float *dbias = nullptr, float *work = nullptr) {
     bool empty = false;
-    sigattn_status s = check_shape(Z, L, H, D, dtype, &empty);
+    sigattn_status s = check_lengths(Z, Lq, Lk, H, D, dtype, &empty);
     if (s != SIGATTN_OK) return s;
     if (empty) return SIGATTN_OK;
     if (!q || !k || !v || !dout || !seqlens_q || !seqlens_k) return SIGATTN_ERR_INVALID_ARG;
@@ -198,53 +216,55 @@ sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void 
                     nullptr,                          static_cast<float *>(dq),
                     static_cast<float *>(dk),         static_cast<float *>(dv),
                     seqlens_q,                        seqlens_k,
-                    Z, L, H, alpha, bias, status, bias_z, db_part};
-        const int64_t rows = static_cast<int64_t>(Z) * L * H;
+                    Z, Lq, Lk, H, alpha, bias, status, bias_z, db_part};
+        const int64_t rows = static_cast<int64_t>(Z) * Lq * H;
+        const int64_t rows_kv = static_cast<int64_t>(Z) * Lk * H;
         dim3 grid(static_cast<unsigned>((rows + 7) / 8));
+        dim3 grid_kv(static_cast<unsigned>((rows_kv + 7) / 8));
         if (parts & kPartDq) {
             s = D == 64 ? launch(f32_dq_kernel<64>, grid, dim3(256), 0, st, p)
                         : launch(f32_dq_kernel<128>, grid, dim3(256), 0, st, p);
             if (s != SIGATTN_OK) return s;
         }
         if (parts & kPartDkdv) {
-            s = D == 64 ? launch(f32_dkdv_kernel<64>, grid, dim3(256), 0, st, p)
-                        : launch(f32_dkdv_kernel<128>, grid, dim3(256), 0, st, p);
+            s = D == 64 ? launch(f32_dkdv_kernel<64>, grid_kv, dim3(256), 0, st, p)
+                        : launch(f32_dkdv_kernel<128>, grid_kv, dim3(256), 0, st, p);
             if (s != SIGATTN_OK) return s;
         }
         if (dbias)
             return launch(dbias_reduce_kernel, dim3(Z), dim3(256), 0, st, static_cast<const float *>(db_part),
-                          dbias_partials_per_sample(L, H, dtype), dbias);
+                          dbias_partials_per_sample(Lq, H, dtype), dbias);
         return SIGATTN_OK;
     }
     if (cc != 100) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
     if ((s = get_encoder()) != SIGATTN_OK) return s;
     CUtensorMap mq, mk, mv, mdo;
-    if ((s = encode_bf16_map(&mq, q, Z, L, H, D)) != SIGATTN_OK) return s;
-    if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
-    if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
-    if ((s = encode_bf16_map(&mdo, dout, Z, L, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mq, q, Z, Lq, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mk, k, Z, Lk, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mv, v, Z, Lk, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mdo, dout, Z, Lq, H, D)) != SIGATTN_OK) return s;
     BwdParams p{static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
-                static_cast<__nv_bfloat16 *>(dv), seqlens_q, seqlens_k, L, H, alpha, bias, status,
+                static_cast<__nv_bfloat16 *>(dv), seqlens_q, seqlens_k, Lq, Lk, H, alpha, bias, status,
                 g_timeout_ns.load(), bias_z, db_part};
     const int mode = g_sigmoid_mode.load();
     if (D == 128)
-        s = mode == kSigmoidTanh ? bwd_bf16<128, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, L, H, parts, st)
-                                 : bwd_bf16<128, kSigmoidExp>(mq, mk, mv, mdo, p, Z, L, H, parts, st);
+        s = mode == kSigmoidTanh ? bwd_bf16<128, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, st)
+                                 : bwd_bf16<128, kSigmoidExp>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, st);
     else
-        s = mode == kSigmoidTanh ? bwd_bf16<64, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, L, H, parts, st)
-                                 : bwd_bf16<64, kSigmoidExp>(mq, mk, mv, mdo, p, Z, L, H, parts, st);
+        s = mode == kSigmoidTanh ? bwd_bf16<64, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, st)
+                                 : bwd_bf16<64, kSigmoidExp>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, st);
     if (s != SIGATTN_OK || !dbias) return s;
     return launch(dbias_reduce_kernel, dim3(Z), dim3(256), 0, st, static_cast<const float *>(db_part),
-                  dbias_partials_per_sample(L, H, dtype), dbias);
+                  dbias_partials_per_sample(Lq, H, dtype), dbias);
 }
 
 // Shared body of sigattn_fwd and sigattn_fwd_bias.
 sigattn_status fwd_impl(const void *q, const void *k, const void *v, void *o,
-                        const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int L, int H,
-                        int D, float alpha, float bias, const float *bias_z, sigattn_dtype dtype,
-                        void *stream) {
+                        const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int Lq,
+                        int Lk, int H, int D, float alpha, float bias, const float *bias_z,
+                        sigattn_dtype dtype, void *stream) {
     bool empty = false;
-    sigattn_status s = check_shape(Z, L, H, D, dtype, &empty);
+    sigattn_status s = check_lengths(Z, Lq, Lk, H, D, dtype, &empty);
     if (s != SIGATTN_OK) return s;
     if (empty) return SIGATTN_OK;
     if (!q || !k || !v || !o || !seqlens_q || !seqlens_k) return SIGATTN_ERR_INVALID_ARG;
@@ -257,9 +277,9 @@ sigattn_status fwd_impl(const void *q, const void *k, const void *v, void *o,
     if (dtype == SIGATTN_FP32) {
         F32Params p{static_cast<const float *>(q), static_cast<const float *>(k),
                     static_cast<const float *>(v), nullptr, static_cast<float *>(o), nullptr,
-                    nullptr, nullptr, seqlens_q, seqlens_k, Z, L, H, alpha, bias, status,
+                    nullptr, nullptr, seqlens_q, seqlens_k, Z, Lq, Lk, H, alpha, bias, status,
                     bias_z, nullptr};
-        const int64_t rows = static_cast<int64_t>(Z) * L * H;
+        const int64_t rows = static_cast<int64_t>(Z) * Lq * H;
         dim3 grid(static_cast<unsigned>((rows + 7) / 8));
         return D == 64 ? launch(f32_fwd_kernel<64>, grid, dim3(256), 0, st, p)
                        : launch(f32_fwd_kernel<128>, grid, dim3(256), 0, st, p);
@@ -267,17 +287,17 @@ sigattn_status fwd_impl(const void *q, const void *k, const void *v, void *o,
     if (cc != 100) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
     if ((s = get_encoder()) != SIGATTN_OK) return s;
     CUtensorMap mq, mk, mv;
-    if ((s = encode_bf16_map(&mq, q, Z, L, H, D)) != SIGATTN_OK) return s;
-    if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
-    if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
-    FwdParams p{static_cast<__nv_bfloat16 *>(o), seqlens_q, seqlens_k, L, H, alpha, bias, status,
-                g_timeout_ns.load(), bias_z};
+    if ((s = encode_bf16_map(&mq, q, Z, Lq, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mk, k, Z, Lk, H, D)) != SIGATTN_OK) return s;
+    if ((s = encode_bf16_map(&mv, v, Z, Lk, H, D)) != SIGATTN_OK) return s;
+    FwdParams p{static_cast<__nv_bfloat16 *>(o), seqlens_q, seqlens_k, Lq, Lk, H, alpha, bias,
+                status, g_timeout_ns.load(), bias_z};
     const int mode = g_sigmoid_mode.load();
     if (D == 128)
-        return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
-                                    : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
-    return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
-                                : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
+        return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, Z, Lq, H, st)
+                                    : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, Z, Lq, H, st);
+    return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, Z, Lq, H, st)
+                                : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, Z, Lq, H, st);
 }
 
 }  // namespace
@@ -287,7 +307,7 @@ extern "C" {
 sigattn_status sigattn_fwd(const void *q, const void *k, const void *v, void *o,
                            const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int L, int H,
                            int D, float alpha, float bias, sigattn_dtype dtype, void *stream) {
-    return fwd_impl(q, k, v, o, seqlens_q, seqlens_k, Z, L, H, D, alpha, bias, nullptr, dtype,
+    return fwd_impl(q, k, v, o, seqlens_q, seqlens_k, Z, L, L, H, D, alpha, bias, nullptr, dtype,
                     stream);
 }
 
@@ -296,7 +316,8 @@ sigattn_status sigattn_fwd_bias(const void *q, const void *k, const void *v, voi
                                 int H, int D, float alpha, const float *bias, sigattn_dtype dtype,
                                 void *stream) {
     if (!bias && Z > 0) return SIGATTN_ERR_INVALID_ARG;
-    return fwd_impl(q, k, v, o, seqlens_q, seqlens_k, Z, L, H, D, alpha, 0.0f, bias, dtype, stream);
+    return fwd_impl(q, k, v, o, seqlens_q, seqlens_k, Z, L, L, H, D, alpha, 0.0f, bias, dtype,
+                    stream);
 }
 
 size_t sigattn_dbias_workspace_bytes(int Z, int L, int H, sigattn_dtype dtype) {
@@ -316,7 +337,7 @@ sigattn_status sigattn_bwd_bias(const void *q, const void *k, const void *v, con
             (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
             return SIGATTN_ERR_INVALID_ARG;
     }
-    return bwd_impl(q, k, v, dout, dq, dk, dv, seqlens_q, seqlens_k, Z, L, H, D, alpha, 0.0f, dtype,
+    return bwd_impl(q, k, v, dout, dq, dk, dv, seqlens_q, seqlens_k, Z, L, L, H, D, alpha, 0.0f, dtype,
                     stream, kPartDq | kPartDkdv, bias, dbias, static_cast<float *>(workspace));
 }
 
@@ -324,7 +345,7 @@ sigattn_status sigattn_bwd(const void *q, const void *k, const void *v, const vo
                            void *dk, void *dv, const int32_t *seqlens_q, const int32_t *seqlens_k,
                            int Z, int L, int H, int D, float alpha, float bias,
                            sigattn_dtype dtype, void *stream) {
-    return bwd_impl(q, k, v, dout, dq, dk, dv, seqlens_q, seqlens_k, Z, L, H, D, alpha, bias, dtype,
+    return bwd_impl(q, k, v, dout, dq, dk, dv, seqlens_q, seqlens_k, Z, L, L, H, D, alpha, bias, dtype,
                     stream, kPartDq | kPartDkdv);
 }
 
@@ -332,7 +353,7 @@ sigattn_status sigattn_bwd_dq(const void *q, const void *k, const void *v, const
                               void *dq, const int32_t *seqlens_q, const int32_t *seqlens_k, int Z,
                               int L, int H, int D, float alpha, float bias, sigattn_dtype dtype,
                               void *stream) {
-    return bwd_impl(q, k, v, dout, dq, nullptr, nullptr, seqlens_q, seqlens_k, Z, L, H, D, alpha,
+    return bwd_impl(q, k, v, dout, dq, nullptr, nullptr, seqlens_q, seqlens_k, Z, L, L, H, D, alpha,
                     bias, dtype, stream, kPartDq);
 }
 
@@ -340,8 +361,24 @@ sigattn_status sigattn_bwd_dkdv(const void *q, const void *k, const void *v, con
                                 void *dk, void *dv, const int32_t *seqlens_q,
                                 const int32_t *seqlens_k, int Z, int L, int H, int D, float alpha,
                                 float bias, sigattn_dtype dtype, void *stream) {
-    return bwd_impl(q, k, v, dout, nullptr, dk, dv, seqlens_q, seqlens_k, Z, L, H, D, alpha, bias,
+    return bwd_impl(q, k, v, dout, nullptr, dk, dv, seqlens_q, seqlens_k, Z, L, L, H, D, alpha, bias,
                     dtype, stream, kPartDkdv);
+}
+
+sigattn_status sigattn_fwd_rect(const void *q, const void *k, const void *v, void *o,
+                                const int32_t *seqlens_q, const int32_t *seqlens_k, int Z, int Lq,
+                                int Lk, int H, int D, float alpha, float bias, sigattn_dtype dtype,
+                                void *stream) {
+    return fwd_impl(q, k, v, o, seqlens_q, seqlens_k, Z, Lq, Lk, H, D, alpha, bias, nullptr, dtype,
+                    stream);
+}
+
+sigattn_status sigattn_bwd_rect(const void *q, const void *k, const void *v, const void *dout,
+                                void *dq, void *dk, void *dv, const int32_t *seqlens_q,
+                                const int32_t *seqlens_k, int Z, int Lq, int Lk, int H, int D,
+                                float alpha, float bias, sigattn_dtype dtype, void *stream) {
+    return bwd_impl(q, k, v, dout, dq, dk, dv, seqlens_q, seqlens_k, Z, Lq, Lk, H, D, alpha, bias,
+                    dtype, stream, kPartDq | kPartDkdv);
 }
 
 sigattn_status sigattn_set_sigmoid_mode(sigattn_sigmoid_mode mode) {
@@ -500,7 +537,7 @@ sigattn_status sigattn_fwd_noalloc(const void *q, const void *k, const void *v, 
     if (dtype == SIGATTN_FP32) {
         F32Params p{static_cast<const float *>(q), static_cast<const float *>(k),
                     static_cast<const float *>(v), nullptr, static_cast<float *>(o), nullptr,
-                    nullptr, nullptr, nq, nk, Z, L, H, alpha, bias, status};
+                    nullptr, nullptr, nq, nk, Z, L, L, H, alpha, bias, status};
         const int64_t rows = static_cast<int64_t>(Z) * L * H;
         dim3 grid(static_cast<unsigned>((rows + 7) / 8));
         return D == 64 ? launch(f32_fwd_kernel<64>, grid, dim3(256), 0, st, p)
@@ -511,7 +548,7 @@ sigattn_status sigattn_fwd_noalloc(const void *q, const void *k, const void *v, 
     if ((s = encode_bf16_map(&mq, q, Z, L, H, D)) != SIGATTN_OK) return s;
     if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
     if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
-    FwdParams p{static_cast<__nv_bfloat16 *>(o), nq, nk, L, H, alpha, bias, status,
+    FwdParams p{static_cast<__nv_bfloat16 *>(o), nq, nk, L, L, H, alpha, bias, status,
                 g_timeout_ns.load(), nullptr};
     const int mode = g_sigmoid_mode.load();
     if (D == 128)

@@ -107,6 +107,20 @@ def test_bias_entry_points_host_validation(lib):
                                 None, 0, None) == 0
 
 
+def test_rect_entry_points_host_validation(lib):
+    vp = ctypes.c_void_p
+    dummy = vp(16)
+    # exactly one of Lq, Lk zero is rejected; both zero is an empty problem
+    assert lib.sigattn_fwd_rect(dummy, dummy, dummy, dummy, dummy, dummy, 1, 128, 0, 1, 64, 1.0,
+                                0.0, 0, None) == 1
+    assert lib.sigattn_bwd_rect(dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy, 1,
+                                0, 128, 1, 64, 1.0, 0.0, 0, None) == 1
+    assert lib.sigattn_fwd_rect(dummy, dummy, dummy, dummy, dummy, dummy, 1, 0, 0, 1, 64, 1.0,
+                                0.0, 0, None) == 0
+    assert lib.sigattn_fwd_rect(dummy, dummy, dummy, dummy, dummy, dummy, 1, 128, 256, 1, 96,
+                                1.0, 0.0, 0, None) == 2
+
+
 def test_no_cpu_fallback(lib):
     import torch
     import padding_aware_sigmoid_b200 as sa
