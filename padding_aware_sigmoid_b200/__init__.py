@@ -22,7 +22,8 @@ __all__ = [
     "last_device_status", "set_wait_timeout_ns", "selftest_wait_timeout", "status_string",
     "version", "library_path", "load_library", "SIGMOID_TANH", "SIGMOID_EXP", "EXPORTS",
     "SigmoidAttention", "bwd_dq", "bwd_dkdv", "last_cuda_error", "fwd_noalloc", "NOALLOC_MAX_Z",
-    "fwd_bias", "bwd_bias", "dbias_workspace_bytes", "fwd_rect", "bwd_rect",
+    "fwd_bias", "bwd_bias", "dbias_workspace_bytes", "fwd_rect", "bwd_rect", "fwd_bwd_host",
+    "fwd_bwd_host_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -50,7 +51,8 @@ EXPORTS = (
     "sigattn_last_device_status", "sigattn_set_wait_timeout_ns", "sigattn_selftest_wait_timeout",
     "sigattn_last_cuda_error", "sigattn_status_string", "sigattn_version",
     "sigattn_fwd_noalloc", "sigattn_fwd_bias", "sigattn_bwd_bias", "sigattn_dbias_workspace_bytes",
-    "sigattn_fwd_rect", "sigattn_bwd_rect",
+    "sigattn_fwd_rect", "sigattn_bwd_rect", "sigattn_fwd_bwd_host",
+    "sigattn_fwd_bwd_host_workspace_bytes",
 )
 
 
@@ -87,6 +89,11 @@ def load_library():
         lib.sigattn_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, cf,
                                          ci, vp]
         lib.sigattn_bwd_dkdv.restype = ci
+        lib.sigattn_fwd_bwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                             cf, cf, ci, vp, ctypes.c_size_t, vp]
+        lib.sigattn_fwd_bwd_host.restype = ci
+        lib.sigattn_fwd_bwd_host_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+        lib.sigattn_fwd_bwd_host_workspace_bytes.restype = ctypes.c_size_t
         lib.sigattn_fwd_rect.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, cf, ci, vp]
         lib.sigattn_fwd_rect.restype = ci
         lib.sigattn_bwd_rect.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf,
@@ -262,6 +269,59 @@ def bwd_rect(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, dq=
         dv.data_ptr(), seqlens_q.data_ptr(), seqlens_k.data_ptr(), Z, Lq, Lk, H, D, float(alpha),
         float(bias), _dtype_code(q), _stream_ptr(q)), "sigattn_bwd_rect")
     return dq, dk, dv
+
+
+def fwd_bwd_host_workspace_bytes(Z: int, L: int, H: int, D: int, dtype) -> int:
+    import torch
+    code = _FP32 if dtype == torch.float32 else _BF16
+    return int(load_library().sigattn_fwd_bwd_host_workspace_bytes(int(Z), int(L), int(H),
+                                                                    int(D), code))
+
+
+def fwd_bwd_host(q, k, v, dout, seqlens_q, seqlens_k, alpha: float, bias: float, outs=None,
+                 workspace=None, device=None):
+    """Forward and backward of a batch held in host memory (CPU tensors, pinned
+    for the copies to overlap the compute): returns host (O, dQ, dK, dV).  Lengths
+    are host int32 [Z] arrays or CPU tensors.  ``workspace``: a device uint8 tensor
+    of at least fwd_bwd_host_workspace_bytes(...) bytes (allocated here when
+    omitted).  The work runs on ``device``'s current stream (default: the current
+    device) and is complete once that stream has passed it."""
+    import numpy as np
+    import torch
+    tensors = [q, k, v, dout]
+    ref = q
+    for t in tensors:
+        if t.is_cuda or t.shape != ref.shape or t.dtype != ref.dtype or not t.is_contiguous():
+            raise ValueError("fwd_bwd_host takes contiguous CPU tensors of one shape and dtype")
+    if outs is None:
+        outs = [torch.empty_like(ref, pin_memory=ref.is_pinned()) for _ in range(4)]
+    nq = np.ascontiguousarray(np.asarray(seqlens_q, dtype=np.int32).reshape(-1))
+    nk = np.ascontiguousarray(np.asarray(seqlens_k, dtype=np.int32).reshape(-1))
+    Z, L, H, D = (int(x) for x in ref.shape)
+    if nq.shape[0] != Z or nk.shape[0] != Z:
+        raise ValueError("seqlens must have Z entries")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    need = fwd_bwd_host_workspace_bytes(Z, L, H, D, ref.dtype)
+    if workspace is None:
+        # kept for later calls: the library's copy streams may still use it after
+        # this call returns, so it is never handed back to the allocator
+        key = (dev.index, need)
+        workspace = _host_workspaces.get(key)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+            _host_workspaces[key] = workspace
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        _check(load_library().sigattn_fwd_bwd_host(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), outs[0].data_ptr(),
+            outs[1].data_ptr(), outs[2].data_ptr(), outs[3].data_ptr(),
+            nq.ctypes.data, nk.ctypes.data, Z, L, H, D, float(alpha), float(bias),
+            _dtype_code(ref), workspace.data_ptr(), workspace.numel(), stream),
+            "sigattn_fwd_bwd_host")
+    return tuple(outs)
+
+
+_host_workspaces = {}
 
 
 def _check_bias(bias, ref):

@@ -39,6 +39,42 @@ sigattn_status cuda_fail(cudaError_t e = cudaSuccess) {
 }
 
 // Current device, its compute capability and its status word.
+// Writes one sample's two lengths into device memory; the values travel as
+// kernel arguments, so nothing is read from host memory after the call returns.
+__global__ void store_lengths_kernel(int32_t *dst, int32_t nq, int32_t nk) {
+    dst[0] = nq;
+    dst[1] = nk;
+}
+
+// Copy streams and events of the host-buffer pipeline, created once per device
+// on first use and kept until process exit (no per-call allocation).
+struct HostPipe {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, in_done[2] = {}, comp_done[2] = {}, freed[2] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+
+sigattn_status device_state(int *dev, int *cc_major, int **status);
+
+sigattn_status host_pipe(int dev, HostPipe **hp) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    HostPipe &p = g_pipe[dev];
+    if (p.in == nullptr) {
+        const unsigned ef = cudaEventDisableTiming;
+        if (cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&p.start, ef) != cudaSuccess)
+            return cuda_fail();
+        for (int i = 0; i < 2; ++i)
+            if (cudaEventCreateWithFlags(&p.in_done[i], ef) != cudaSuccess ||
+                cudaEventCreateWithFlags(&p.comp_done[i], ef) != cudaSuccess ||
+                cudaEventCreateWithFlags(&p.freed[i], ef) != cudaSuccess)
+                return cuda_fail();
+    }
+    *hp = &p;
+    return SIGATTN_OK;
+}
+
 sigattn_status device_state(int *dev, int *cc_major, int **status) {
     cudaError_t e = cudaGetDevice(dev);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -379,6 +415,90 @@ sigattn_status sigattn_bwd_rect(const void *q, const void *k, const void *v, con
                                 float alpha, float bias, sigattn_dtype dtype, void *stream) {
     return bwd_impl(q, k, v, dout, dq, dk, dv, seqlens_q, seqlens_k, Z, Lq, Lk, H, D, alpha, bias,
                     dtype, stream, kPartDq | kPartDkdv);
+}
+
+size_t sigattn_fwd_bwd_host_workspace_bytes(int Z, int L, int H, int D, sigattn_dtype dtype) {
+    if (Z <= 0 || L <= 0 || H <= 0 || (D != 64 && D != 128)) return 0;
+    if (dtype != SIGATTN_BF16 && dtype != SIGATTN_FP32) return 0;
+    const size_t per = static_cast<size_t>(L) * H * D * (dtype == SIGATTN_BF16 ? 2 : 4);
+    // two sample slots of eight tensors, then two 256-byte length records
+    return 2 * 8 * per + 2 * 256;
+}
+
+sigattn_status sigattn_fwd_bwd_host(const void *q, const void *k, const void *v, const void *dout,
+                                    void *o, void *dq, void *dk, void *dv,
+                                    const int32_t *host_seqlens_q, const int32_t *host_seqlens_k,
+                                    int Z, int L, int H, int D, float alpha, float bias,
+                                    sigattn_dtype dtype, void *workspace, size_t workspace_bytes,
+                                    void *stream) {
+    bool empty = false;
+    sigattn_status s = check_shape(Z, L, H, D, dtype, &empty);
+    if (s != SIGATTN_OK) return s;
+    if (empty) return SIGATTN_OK;
+    if (!q || !k || !v || !dout || !o || !dq || !dk || !dv || !host_seqlens_q || !host_seqlens_k)
+        return SIGATTN_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < sigattn_fwd_bwd_host_workspace_bytes(Z, L, H, D, dtype))
+        return SIGATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SIGATTN_ERR_MISALIGNED;
+    for (int z = 0; z < Z; ++z)
+        if (host_seqlens_q[z] < 0 || host_seqlens_q[z] > L || host_seqlens_k[z] < 0 ||
+            host_seqlens_k[z] > L)
+            return SIGATTN_ERR_INVALID_ARG;
+    int dev, cc;
+    int *status;
+    if ((s = device_state(&dev, &cc, &status)) != SIGATTN_OK) return s;
+    HostPipe *hp;
+    if ((s = host_pipe(dev, &hp)) != SIGATTN_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t per = static_cast<size_t>(L) * H * D * (dtype == SIGATTN_BF16 ? 2 : 4);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const void *hin[4] = {q, k, v, dout};
+    void *hout[4] = {o, dq, dk, dv};
+    // the copy streams start after the caller's earlier work on `stream`
+    if (cudaEventRecord(hp->start, st) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
+        return cuda_fail();
+    for (int z = 0; z < Z; ++z) {
+        const int slot = z & 1;
+        uint8_t *base = ws + static_cast<size_t>(slot) * 8 * per;
+        int32_t *lens = reinterpret_cast<int32_t *>(ws + 16 * per + slot * 256);
+        // inputs of sample z: the slot is free once sample z-2's outputs are read back
+        if (z >= 2 && cudaStreamWaitEvent(hp->in, hp->freed[slot], 0) != cudaSuccess)
+            return cuda_fail();
+        if ((s = launch(store_lengths_kernel, dim3(1), dim3(1), 0, hp->in, lens,
+                        static_cast<int32_t>(host_seqlens_q[z]),
+                        static_cast<int32_t>(host_seqlens_k[z]))) != SIGATTN_OK)
+            return s;
+        for (int t = 0; t < 4; ++t)
+            if (cudaMemcpyAsync(base + t * per, static_cast<const uint8_t *>(hin[t]) + z * per, per,
+                                cudaMemcpyHostToDevice, hp->in) != cudaSuccess)
+                return cuda_fail();
+        if (cudaEventRecord(hp->in_done[slot], hp->in) != cudaSuccess ||
+            cudaStreamWaitEvent(st, hp->in_done[slot], 0) != cudaSuccess)
+            return cuda_fail();
+        // forward and backward of sample z on the caller's stream
+        s = fwd_impl(base, base + per, base + 2 * per, base + 4 * per, lens, lens + 1, 1, L, L, H, D,
+                     alpha, bias, nullptr, dtype, stream);
+        if (s != SIGATTN_OK) return s;
+        s = bwd_impl(base, base + per, base + 2 * per, base + 3 * per, base + 5 * per,
+                     base + 6 * per, base + 7 * per, lens, lens + 1, 1, L, L, H, D, alpha, bias,
+                     dtype, stream, kPartDq | kPartDkdv);
+        if (s != SIGATTN_OK) return s;
+        if (cudaEventRecord(hp->comp_done[slot], st) != cudaSuccess ||
+            cudaStreamWaitEvent(hp->out, hp->comp_done[slot], 0) != cudaSuccess)
+            return cuda_fail();
+        // outputs of sample z back to the host while the next sample computes
+        for (int t = 0; t < 4; ++t)
+            if (cudaMemcpyAsync(static_cast<uint8_t *>(hout[t]) + z * per, base + (4 + t) * per, per,
+                                cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+                return cuda_fail();
+        if (cudaEventRecord(hp->freed[slot], hp->out) != cudaSuccess) return cuda_fail();
+    }
+    // the call completes on `stream` once every output has reached the host
+    for (int slot = 0; slot < (Z > 1 ? 2 : 1); ++slot)
+        if (cudaStreamWaitEvent(st, hp->freed[slot], 0) != cudaSuccess) return cuda_fail();
+    return SIGATTN_OK;
 }
 
 sigattn_status sigattn_set_sigmoid_mode(sigattn_sigmoid_mode mode) {
