@@ -244,18 +244,25 @@ def test_autograd_module_matches_oracle():
 
 
 
+@pytest.mark.parametrize("mode", ["tanh", "exp"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_long_sequence_sampled(D):
+def test_long_sequence_sampled(D, mode):
     """L = 65536 (4x the headline length) with one full and one ragged sample:
-    sampled rows of every output against the oracle (index arithmetic beyond
-    2^31 elements per tensor row range, deepest loops)."""
+    sampled rows of every output against the oracle (the deepest key loops and
+    the most negative bias, b = -ln 65536, where the tanh form's left-tail error
+    is largest)."""
     dev = _dev()
     Z, L, H = 2, 65536, 1
     n = (65536, 40001)
     inp = _case(Z, L, H, D, n, n, seed=4000 + D)
-    outs = _run(inp, dev)
+    old = sa.get_sigmoid_mode()
+    sa.set_sigmoid_mode(sa.SIGMOID_TANH if mode == "tanh" else sa.SIGMOID_EXP)
+    try:
+        outs = _run(inp, dev)
+    finally:
+        sa.set_sigmoid_mode(old)
     rep = _check_sampled(inp, outs, 12, seed=40 + D)
-    print(f"L=65536 D={D}: max-abs/max|ref| / L1 rel:",
+    print(f"L=65536 D={D} sigma {mode}: max-abs/max|ref| / L1 rel:",
           {k: ("%.2e/%.2e" % v) for k, v in rep.items()})
 
 
