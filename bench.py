@@ -332,6 +332,31 @@ def our_arm(args, world, rank, local):
     del inp4
     torch.cuda.empty_cache()
 
+    # each kernel also timed on its own (10 back-to-back launches after the step
+    # loop): the GPU's power-limited clock then follows that kernel alone
+    import torch as _t
+    inp3 = make_device_inputs(w3, device, rank)
+    o_, dq_, dk_, dv_ = (_t.empty_like(inp3["q"]) for _ in range(4))
+    a3 = (inp3["q"], inp3["k"], inp3["v"])
+    alone = {}
+    for name, call in (
+            ("fwd", lambda: sa.fwd(*a3, inp3["nq"], inp3["nk"], w3.alpha, w3.bias, out=o_)),
+            ("bwd_dq", lambda: sa.bwd_dq(*a3, inp3["dout"], inp3["nq"], inp3["nk"], w3.alpha,
+                                         w3.bias, dq=dq_)),
+            ("bwd_dkdv", lambda: sa.bwd_dkdv(*a3, inp3["dout"], inp3["nq"], inp3["nk"], w3.alpha,
+                                             w3.bias, dk=dk_, dv=dv_))):
+        for _ in range(3):
+            call()
+        st_ = _t.cuda.current_stream(device)
+        e0, e1 = _t.cuda.Event(enable_timing=True), _t.cuda.Event(enable_timing=True)
+        e0.record(st_)
+        for _ in range(10):
+            call()
+        e1.record(st_)
+        _t.cuda.synchronize(device)
+        alone[name] = e0.elapsed_time(e1) / 10
+    del inp3, o_, dq_, dk_, dv_
+
     # the D = 64 workloads (2: short ragged sequences, 5: lognormal lengths, large
     # scores), timed the same way with their own valid-FLOP counts
     d64 = {}
@@ -409,6 +434,13 @@ def our_arm(args, world, rank, local):
         "fwd_tflops": fwd_tf,
         "bwd_tflops": bwd_tf,
         "fwd_ms": fwd_ms, "bwd_dq_ms": dq_ms, "bwd_dkdv_ms": dkdv_ms,
+        "alone": {
+            "note": "each kernel launched 10x back to back on its own, outside the step loop",
+            "fwd_ms": alone["fwd"], "bwd_dq_ms": alone["bwd_dq"],
+            "bwd_dkdv_ms": alone["bwd_dkdv"],
+            "fwd_tflops": f3 / (alone["fwd"] * 1e-3) / 1e12,
+            "bwd_tflops": 2.5 * f3 / ((alone["bwd_dq"] + alone["bwd_dkdv"]) * 1e-3) / 1e12,
+        },
         "fwd_pct_of_peak": 100.0 * fwd_tf / pk["bf16"],
         "bwd_pct_of_peak": 100.0 * bwd_tf / pk["bf16"],
         "pad25": {
