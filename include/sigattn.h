@@ -274,6 +274,20 @@ const char *sigattn_last_cuda_error(void);
 /* Human-readable name of a status code (static string). */
 const char *sigattn_status_string(sigattn_status s);
 
+/* Order in which the bf16 kernels start the samples of a batch: blocks are
+ * dispatched in grid order, and the block of grid position z works on the
+ * sample of rank z by decreasing work, ties by increasing index, so the
+ * samples with the most tiles start first and the short ones fill in behind
+ * them.  A sample's work is its key length n_k (forward, dQ kernel) or its
+ * query length n_q (dK/dV kernel), and 0 when its other length is 0.  For
+ * Z > 64 the kernels keep the index order.
+ *
+ * This host function applies the same rule: work is host int32[Z], order
+ * (host int32[Z], written) receives the sample index for each rank.  It runs
+ * no device code.  Returns SIGATTN_ERR_INVALID_ARG for a NULL pointer or
+ * Z < 0. */
+sigattn_status sigattn_launch_order(const int32_t *work, int Z, int32_t *order);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int sigattn_version(void);
 

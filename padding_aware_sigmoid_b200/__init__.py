@@ -23,7 +23,7 @@ __all__ = [
     "version", "library_path", "load_library", "SIGMOID_TANH", "SIGMOID_EXP", "EXPORTS",
     "SigmoidAttention", "bwd_dq", "bwd_dkdv", "last_cuda_error", "fwd_noalloc", "NOALLOC_MAX_Z",
     "fwd_bias", "bwd_bias", "dbias_workspace_bytes", "fwd_rect", "bwd_rect", "fwd_bwd_host",
-    "fwd_bwd_host_workspace_bytes",
+    "fwd_bwd_host_workspace_bytes", "launch_order",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -52,7 +52,7 @@ EXPORTS = (
     "sigattn_last_cuda_error", "sigattn_status_string", "sigattn_version",
     "sigattn_fwd_noalloc", "sigattn_fwd_bias", "sigattn_bwd_bias", "sigattn_dbias_workspace_bytes",
     "sigattn_fwd_rect", "sigattn_bwd_rect", "sigattn_fwd_bwd_host",
-    "sigattn_fwd_bwd_host_workspace_bytes",
+    "sigattn_fwd_bwd_host_workspace_bytes", "sigattn_launch_order",
 )
 
 
@@ -123,6 +123,8 @@ def load_library():
         lib.sigattn_status_string.argtypes = [ci]
         lib.sigattn_status_string.restype = ctypes.c_char_p
         lib.sigattn_version.restype = ci
+        lib.sigattn_launch_order.argtypes = [vp, ci, vp]
+        lib.sigattn_launch_order.restype = ci
         _lib = lib
         return lib
 
@@ -462,6 +464,17 @@ def status_string(code: int) -> str:
 
 def version() -> int:
     return int(load_library().sigattn_version())
+
+
+def launch_order(work) -> list:
+    """Sample index for each launch rank: decreasing work, ties by index (the
+    rule the bf16 kernels use to start long samples first)."""
+    import numpy as np
+    w = np.ascontiguousarray(np.asarray(work, dtype=np.int32))
+    order = np.empty(w.shape[0], dtype=np.int32)
+    _check(load_library().sigattn_launch_order(w.ctypes.data, int(w.shape[0]),
+                                               order.ctypes.data), "sigattn_launch_order")
+    return order.tolist()
 
 
 from .autograd import SigmoidAttention  # noqa: E402  (needs the functions above)

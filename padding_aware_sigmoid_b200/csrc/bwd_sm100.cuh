@@ -63,7 +63,8 @@ struct BwdLayout {
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
     static constexpr int OFF_RED = OFF_ABORT + 8;      // 8 floats: per-warp db partials
-    static constexpr int SMEM_ALLOC = OFF_RED + 32 + 1024;
+    static constexpr int OFF_SAMPLE = OFF_RED + 32;    // this block's sample and lengths
+    static constexpr int SMEM_ALLOC = OFF_SAMPLE + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
     static_assert(COL_ACC1 + D <= TMEM_COLS, "TMEM budget");
@@ -177,17 +178,10 @@ __global__ void __launch_bounds__(384, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
     const int warp = warp_id(), lane = lane_id();
-    const int z = blockIdx.z, h = blockIdx.y, qtile = blockIdx.x;
-    const int L = p.Lq;     // rows of this kernel's tiles and outputs: queries
-    int nq = p.seqlens_q[z], nk = p.seqlens_k[z];
-    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
-        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
-        nq = min(max(nq, 0), L);
-        nk = min(max(nk, 0), p.Lk);
-    }
-    const int nkv = (nk + 127) / 128;
-    const bool work = qtile * 128 < nq && nkv > 0;
 
+    // samples start by decreasing key length: warp 0 picks this block's sample
+    BlockSample *sample_slot = reinterpret_cast<BlockSample *>(smem + Lay::OFF_SAMPLE);
+    if (warp == 0) publish_block_sample(p.seqlens_q, p.seqlens_k, true, sample_slot);
     if (threadIdx.x == 0) {
         mbar_init(res_full, 1);
         for (int s = 0; s < SX; ++s) {
@@ -224,6 +218,18 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
+
+    const BlockSample bs = *sample_slot;
+    const int z = bs.z, h = blockIdx.y, qtile = blockIdx.x;
+    const int L = p.Lq;     // rows of this kernel's tiles and outputs: queries
+    int nq = bs.nq, nk = bs.nk;
+    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
+        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
+        nq = min(max(nq, 0), L);
+        nk = min(max(nk, 0), p.Lk);
+    }
+    const int nkv = (nk + 127) / 128;
+    const bool work = qtile * 128 < nq && nkv > 0;
 
     if (warp == 0) {
         if (work && lane == 0) {
@@ -457,17 +463,10 @@ __global__ void __launch_bounds__(384, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
     const int warp = warp_id(), lane = lane_id();
-    const int z = blockIdx.z, h = blockIdx.y, ktile = blockIdx.x;
-    const int L = p.Lk;     // rows of this kernel's tiles and outputs: keys
-    int nq = p.seqlens_q[z], nk = p.seqlens_k[z];
-    if (nq < 0 || nq > p.Lq || nk < 0 || nk > L) {
-        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
-        nq = min(max(nq, 0), p.Lq);
-        nk = min(max(nk, 0), L);
-    }
-    const int nqt = (nq + 127) / 128;
-    const bool work = ktile * 128 < nk && nqt > 0;
 
+    // samples start by decreasing query length: warp 0 picks this block's sample
+    BlockSample *sample_slot = reinterpret_cast<BlockSample *>(smem + Lay::OFF_SAMPLE);
+    if (warp == 0) publish_block_sample(p.seqlens_q, p.seqlens_k, false, sample_slot);
     if (threadIdx.x == 0) {
         mbar_init(res_full, 1);
         for (int s = 0; s < SX; ++s) {
@@ -502,6 +501,18 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
+
+    const BlockSample bs = *sample_slot;
+    const int z = bs.z, h = blockIdx.y, ktile = blockIdx.x;
+    const int L = p.Lk;     // rows of this kernel's tiles and outputs: keys
+    int nq = bs.nq, nk = bs.nk;
+    if (nq < 0 || nq > p.Lq || nk < 0 || nk > L) {
+        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
+        nq = min(max(nq, 0), p.Lq);
+        nk = min(max(nk, 0), L);
+    }
+    const int nqt = (nq + 127) / 128;
+    const bool work = ktile * 128 < nk && nqt > 0;
 
     if (warp == 0) {
         if (work && lane == 0) {

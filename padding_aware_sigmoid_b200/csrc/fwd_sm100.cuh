@@ -63,7 +63,8 @@ struct FwdLayout {
     static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 5;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
-    static constexpr int BYTES = OFF_ABORT + 8;
+    static constexpr int OFF_SAMPLE = OFF_ABORT + 8;   // this block's sample and lengths
+    static constexpr int BYTES = OFF_SAMPLE + 16;
     static constexpr int SMEM_ALLOC = BYTES + 1024;  // slack to align the base to 1 KiB
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -107,20 +108,9 @@ __global__ void __launch_bounds__(384, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
     const int warp = warp_id(), lane = lane_id();
-    const int z = blockIdx.z, h = blockIdx.y;
-    const int qtile0 = blockIdx.x * 2;
-    const int L = p.Lq;     // query rows of this problem (O has the same layout)
-
-    int nq = p.seqlens_q[z], nk = p.seqlens_k[z];
-    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
-        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
-        nq = min(max(nq, 0), L);
-        nk = min(max(nk, 0), p.Lk);
-    }
-    const int ntiles = (qtile0 * Lay::BM < nq ? 1 : 0) + ((qtile0 + 1) * Lay::BM < nq ? 1 : 0);
-    const int nkv = (nk + Lay::BN - 1) / Lay::BN;
-    const bool work = ntiles > 0 && nkv > 0;
-
+    // samples start by decreasing key length: warp 0 picks this block's sample
+    BlockSample *sample_slot = reinterpret_cast<BlockSample *>(smem + Lay::OFF_SAMPLE);
+    if (warp == 0) publish_block_sample(p.seqlens_q, p.seqlens_k, true, sample_slot);
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < KS; ++s) {
@@ -153,6 +143,20 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
+
+    const BlockSample bs = *sample_slot;
+    const int z = bs.z, h = blockIdx.y;
+    const int qtile0 = blockIdx.x * 2;
+    const int L = p.Lq;     // query rows of this problem (O has the same layout)
+    int nq = bs.nq, nk = bs.nk;
+    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
+        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
+        nq = min(max(nq, 0), L);
+        nk = min(max(nk, 0), p.Lk);
+    }
+    const int ntiles = (qtile0 * Lay::BM < nq ? 1 : 0) + ((qtile0 + 1) * Lay::BM < nq ? 1 : 0);
+    const int nkv = (nk + Lay::BN - 1) / Lay::BN;
+    const bool work = ntiles > 0 && nkv > 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer

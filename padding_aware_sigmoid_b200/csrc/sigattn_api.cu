@@ -581,7 +581,13 @@ const char *sigattn_last_cuda_error(void) {
     return cudaGetErrorString(static_cast<cudaError_t>(e));
 }
 
-int sigattn_version(void) { return 100; }
+sigattn_status sigattn_launch_order(const int32_t *work, int Z, int32_t *order) {
+    if (Z < 0 || (Z > 0 && (!work || !order))) return SIGATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < Z; ++i) order[rank_by_work(i, work, Z)] = i;
+    return SIGATTN_OK;
+}
+
+int sigattn_version(void) { return 101; }
 
 }  // extern "C"
 

@@ -353,6 +353,68 @@ __device__ __forceinline__ void sigma_warps_sync(int count) {
     asm volatile("bar.sync 1, %0;" ::"r"(count) : "memory");
 }
 
+// ------------------------------------------------------------------ launch order
+
+// Sample j (work wj) comes before sample i (work wi) when samples are ordered by
+// decreasing work, ties by increasing index: a stable descending sort.
+__host__ __device__ inline bool ranks_before(int wj, int j, int wi, int i) {
+    return wj > wi || (wj == wi && j < i);
+}
+
+// Position of sample i in that order; over Z samples the positions are a
+// permutation of 0..Z-1.
+__host__ __device__ inline int rank_by_work(int i, const int *work, int Z) {
+    int r = 0;
+    for (int j = 0; j < Z; ++j) r += ranks_before(work[j], j, work[i], i);
+    return r;
+}
+
+// Blocks are dispatched in increasing linear index (x fastest, z slowest), so a
+// grid whose z coordinate runs over the samples starts them in index order, and
+// the blocks of a long sample that comes last run on alone at the end.  Here the
+// block at z = r works on the sample of rank r by decreasing work: the key
+// length n_k (keys_are_work) or the query length n_q, and 0 when the sample's
+// other length is 0.  The longest samples start first and the short ones fill
+// in behind them.
+//
+// One warp finds the sample with shuffles (lane l holds samples l and l + 32)
+// and writes it to `slot` in shared memory; the other warps read it there after
+// the block barrier that ends their setup, so the lookup overlaps the setup and
+// adds no barrier.  All 32 lanes of that warp call it.  The slot holds the
+// sample and its two lengths as stored (range checks stay with the reader).
+// Above kMaxRankedSamples samples the index order is kept.
+struct BlockSample {
+    int z, nq, nk, unused;
+};
+constexpr int kMaxRankedSamples = 64;
+__device__ __forceinline__ void publish_block_sample(const int32_t *seqlens_q,
+                                                     const int32_t *seqlens_k, bool keys_are_work,
+                                                     BlockSample *slot) {
+    const int Z = static_cast<int>(gridDim.z), r = static_cast<int>(blockIdx.z);
+    const int lane = static_cast<int>(threadIdx.x & 31);
+    if (Z > kMaxRankedSamples) {
+        if (lane == 0) *slot = BlockSample{r, seqlens_q[r], seqlens_k[r], 0};
+        return;
+    }
+    int nq[2], nk[2], w[2], rank[2] = {0, 0};
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const int i = lane + 32 * c;
+        nq[c] = i < Z ? seqlens_q[i] : 0;
+        nk[c] = i < Z ? seqlens_k[i] : 0;
+        w[c] = keys_are_work ? (nq[c] > 0 ? nk[c] : 0) : (nk[c] > 0 ? nq[c] : 0);
+    }
+    // only the Z live samples are compared (a short loop for small batches)
+    for (int j = 0; j < Z; ++j) {
+        const int wj = __shfl_sync(0xffffffffu, j < 32 ? w[0] : w[1], j & 31);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) rank[c] += ranks_before(wj, j, w[c], lane + 32 * c);
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+        if (lane + 32 * c < Z && rank[c] == r) *slot = BlockSample{lane + 32 * c, nq[c], nk[c], 0};
+}
+
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 

@@ -75,6 +75,10 @@ SMALL = [
     (2, 520, 2, 128, (513, 128), (520, 255)),
     (1, 1000, 2, 64, (999,), (1000,)),
     (2, 640, 1, 128, (0, 640), (640, 0)),
+    # lengths out of order, ties and empty samples: the kernels start samples by
+    # decreasing length, so grid position and sample index differ here
+    (6, 384, 2, 128, (100, 384, 0, 300, 384, 1), (384, 100, 200, 0, 383, 2)),
+    (5, 256, 2, 64, (17, 256, 256, 129, 3), (256, 5, 256, 100, 256)),
 ]
 
 

@@ -137,3 +137,23 @@ def test_product_path_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
                 assert "sigattn_oracle" not in text, f
+
+
+def test_launch_order_is_a_stable_descending_sort(lib):
+    """The kernels start samples by decreasing work (ties by index); the host
+    entry point applies the same rule, so it is checked here without a GPU."""
+    import numpy as np
+    import padding_aware_sigmoid_b200 as sa
+    assert sa.launch_order([5, 9, 9, 0, 7]) == [1, 2, 4, 0, 3]
+    assert sa.launch_order([]) == []
+    assert sa.launch_order([3, 3, 3]) == [0, 1, 2]
+    g = np.random.default_rng(3)
+    for Z in (1, 2, 7, 64, 384):
+        w = g.integers(0, 40, size=Z).astype(np.int32)
+        want = np.argsort(-w.astype(np.int64), kind="stable").tolist()
+        got = sa.launch_order(w)
+        assert got == want
+        assert sorted(got) == list(range(Z))
+    assert lib.sigattn_launch_order(None, 3, None) == 1
+    assert lib.sigattn_launch_order(None, -1, None) == 1
+    assert lib.sigattn_launch_order(None, 0, None) == 0
