@@ -138,24 +138,29 @@ sigattn_status sigattn_bwd_rect(const void *q, const void *k, const void *v, con
                                 float alpha, float bias, sigattn_dtype dtype, void *stream);
 
 /* Forward and backward of a batch held in HOST memory, with the transfers
- * overlapped: per sample z, q, k, v, dout (host, [Z][L][H][D]) are copied to
- * the device on a library-owned copy stream while sample z-1 computes; the
- * forward and the backward of sample z run on `stream`; o, dq, dk, dv (host,
- * [Z][L][H][D]) are copied back on a second copy stream while sample z+1
- * computes.  The results equal sigattn_fwd + sigattn_bwd on the same data
- * bit for bit (the kernels see one sample at a time, and samples are
- * independent).
+ * overlapped.  The batch is cut into units of one sample and a group of heads
+ * (whole samples once Z >= 8; otherwise about 8 units in all, so that the
+ * first copy in and the last copy out, which nothing overlaps, are short).
+ * Per unit, its rows of q, k, v, dout (host, [Z][L][H][D]) are copied into a
+ * compact device slot on a library-owned copy stream while earlier units
+ * compute; the forward and the backward of the unit run on one of two
+ * library-owned compute streams (consecutive units alternate, so one unit's
+ * last wave overlaps the next unit's first); its o, dq, dk, dv rows go back to
+ * the host tensors on a second copy stream while later units compute.  The
+ * results equal sigattn_fwd + sigattn_bwd on the same data bit for bit (every
+ * (sample, head) pair is computed on its own by the same kernels).
  * host_seqlens_q / host_seqlens_k: int32[Z] in host memory, checked and read
  * on the host during the call (values outside [0, L] are
  * SIGATTN_ERR_INVALID_ARG); they may be reused as soon as it returns.
  * workspace: caller-owned device memory of at least
  * sigattn_fwd_bwd_host_workspace_bytes(Z, L, H, D, dtype) bytes, 256-byte
- * aligned (two sample slots of the eight tensors plus their lengths).
+ * aligned (three unit slots of the eight tensors plus their lengths).
  * The transfers overlap the compute only when the host buffers are pinned
  * (page-locked); pageable buffers work but serialise the copies.  Returns when
- * all work is enqueued; it is complete once `stream` has passed it.  The copy
- * streams are created on the first call on each device and kept; calls on one
- * device must not overlap each other (they share those streams).
+ * all work is enqueued; it is complete once `stream` has passed it (the
+ * pipeline's streams start after the work already on `stream`).  The streams
+ * are created on the first call on each device and kept; calls on one device
+ * must not overlap each other (they share those streams).
  * Errors as sigattn_bwd, plus SIGATTN_ERR_INVALID_ARG for a missing or small
  * workspace and SIGATTN_ERR_MISALIGNED for a misaligned one. */
 sigattn_status sigattn_fwd_bwd_host(const void *q, const void *k, const void *v, const void *dout,

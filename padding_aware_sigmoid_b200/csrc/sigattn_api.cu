@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <mutex>
@@ -46,12 +47,26 @@ __global__ void store_lengths_kernel(int32_t *dst, int32_t nq, int32_t nk) {
     dst[1] = nk;
 }
 
-// Copy streams and events of the host-buffer pipeline, created once per device
-// on first use and kept until process exit (no per-call allocation).
+// Streams and events of the host-buffer pipeline, created once per device on
+// first use and kept until process exit (no per-call allocation): one stream
+// for host-to-device copies, one for device-to-host copies, and two compute
+// streams so that consecutive units' kernels overlap where one unit's last
+// wave leaves SMs idle.
+constexpr int kPipeSlots = 3;
 struct HostPipe {
-    cudaStream_t in = nullptr, out = nullptr;
-    cudaEvent_t start = nullptr, in_done[2] = {}, comp_done[2] = {}, freed[2] = {};
+    cudaStream_t in = nullptr, out = nullptr, comp[2] = {};
+    cudaEvent_t start = nullptr, in_done[kPipeSlots] = {}, comp_done[kPipeSlots] = {},
+                freed[kPipeSlots] = {};
 };
+
+// The pipeline's unit of work: `hc` heads (the last unit of a sample may have
+// fewer) of one sample.  A batch of few samples is split by heads so that the
+// first copy in and the last copy out, which nothing overlaps, are short.
+constexpr int kPipeUnitsTarget = 8;
+int pipe_heads_per_unit(int Z, int H) {
+    const int chunks = std::min(H, (kPipeUnitsTarget + Z - 1) / Z);
+    return (H + chunks - 1) / chunks;
+}
 HostPipe g_pipe[kMaxDevices];
 
 sigattn_status device_state(int *dev, int *cc_major, int **status);
@@ -63,9 +78,11 @@ sigattn_status host_pipe(int dev, HostPipe **hp) {
         const unsigned ef = cudaEventDisableTiming;
         if (cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) != cudaSuccess ||
             cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&p.comp[0], cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&p.comp[1], cudaStreamNonBlocking) != cudaSuccess ||
             cudaEventCreateWithFlags(&p.start, ef) != cudaSuccess)
             return cuda_fail();
-        for (int i = 0; i < 2; ++i)
+        for (int i = 0; i < kPipeSlots; ++i)
             if (cudaEventCreateWithFlags(&p.in_done[i], ef) != cudaSuccess ||
                 cudaEventCreateWithFlags(&p.comp_done[i], ef) != cudaSuccess ||
                 cudaEventCreateWithFlags(&p.freed[i], ef) != cudaSuccess)
@@ -420,9 +437,10 @@ sigattn_status sigattn_bwd_rect(const void *q, const void *k, const void *v, con
 size_t sigattn_fwd_bwd_host_workspace_bytes(int Z, int L, int H, int D, sigattn_dtype dtype) {
     if (Z <= 0 || L <= 0 || H <= 0 || (D != 64 && D != 128)) return 0;
     if (dtype != SIGATTN_BF16 && dtype != SIGATTN_FP32) return 0;
-    const size_t per = static_cast<size_t>(L) * H * D * (dtype == SIGATTN_BF16 ? 2 : 4);
-    // two sample slots of eight tensors, then two 256-byte length records
-    return 2 * 8 * per + 2 * 256;
+    const size_t per = static_cast<size_t>(L) * pipe_heads_per_unit(Z, H) * D *
+                       (dtype == SIGATTN_BF16 ? 2 : 4);
+    // kPipeSlots unit slots of eight tensors, then one 256-byte length record per slot
+    return kPipeSlots * 8 * per + kPipeSlots * 256;
 }
 
 sigattn_status sigattn_fwd_bwd_host(const void *q, const void *k, const void *v, const void *dout,
@@ -450,54 +468,68 @@ sigattn_status sigattn_fwd_bwd_host(const void *q, const void *k, const void *v,
     HostPipe *hp;
     if ((s = host_pipe(dev, &hp)) != SIGATTN_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t per = static_cast<size_t>(L) * H * D * (dtype == SIGATTN_BF16 ? 2 : 4);
+    const size_t es = dtype == SIGATTN_BF16 ? 2 : 4;
+    const int hpu = pipe_heads_per_unit(Z, H);
+    const int chunks = (H + hpu - 1) / hpu;
+    const size_t slot_tensor = static_cast<size_t>(L) * hpu * D * es;   // one tensor of a slot
+    const size_t host_row = static_cast<size_t>(H) * D * es;             // one row of a host tensor
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    const void *hin[4] = {q, k, v, dout};
-    void *hout[4] = {o, dq, dk, dv};
-    // the copy streams start after the caller's earlier work on `stream`
-    if (cudaEventRecord(hp->start, st) != cudaSuccess ||
-        cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
-        return cuda_fail();
-    for (int z = 0; z < Z; ++z) {
-        const int slot = z & 1;
-        uint8_t *base = ws + static_cast<size_t>(slot) * 8 * per;
-        int32_t *lens = reinterpret_cast<int32_t *>(ws + 16 * per + slot * 256);
-        // inputs of sample z: the slot is free once sample z-2's outputs are read back
-        if (z >= 2 && cudaStreamWaitEvent(hp->in, hp->freed[slot], 0) != cudaSuccess)
+    const uint8_t *hin[4] = {static_cast<const uint8_t *>(q), static_cast<const uint8_t *>(k),
+                             static_cast<const uint8_t *>(v), static_cast<const uint8_t *>(dout)};
+    uint8_t *hout[4] = {static_cast<uint8_t *>(o), static_cast<uint8_t *>(dq),
+                        static_cast<uint8_t *>(dk), static_cast<uint8_t *>(dv)};
+    // every pipeline stream starts after the caller's earlier work on `stream`
+    if (cudaEventRecord(hp->start, st) != cudaSuccess) return cuda_fail();
+    for (cudaStream_t x : {hp->in, hp->out, hp->comp[0], hp->comp[1]})
+        if (cudaStreamWaitEvent(x, hp->start, 0) != cudaSuccess) return cuda_fail();
+    const int units = Z * chunks;
+    for (int u = 0; u < units; ++u) {
+        const int z = u / chunks, h0 = (u % chunks) * hpu, hc = std::min(hpu, H - h0);
+        const int slot = u % kPipeSlots;
+        cudaStream_t cs = hp->comp[u & 1];
+        uint8_t *base = ws + static_cast<size_t>(slot) * 8 * slot_tensor;
+        int32_t *lens = reinterpret_cast<int32_t *>(ws + kPipeSlots * 8 * slot_tensor + slot * 256);
+        // rows of this unit: L rows of hc heads, host rows H heads apart
+        const size_t width = static_cast<size_t>(hc) * D * es;
+        const size_t host_off = (static_cast<size_t>(z) * L * H + h0) * D * es;
+        // inputs: the slot is free once unit u - kPipeSlots has been read back
+        if (u >= kPipeSlots && cudaStreamWaitEvent(hp->in, hp->freed[slot], 0) != cudaSuccess)
             return cuda_fail();
         if ((s = launch(store_lengths_kernel, dim3(1), dim3(1), 0, hp->in, lens,
                         static_cast<int32_t>(host_seqlens_q[z]),
                         static_cast<int32_t>(host_seqlens_k[z]))) != SIGATTN_OK)
             return s;
         for (int t = 0; t < 4; ++t)
-            if (cudaMemcpyAsync(base + t * per, static_cast<const uint8_t *>(hin[t]) + z * per, per,
-                                cudaMemcpyHostToDevice, hp->in) != cudaSuccess)
+            if (cudaMemcpy2DAsync(base + t * slot_tensor, width, hin[t] + host_off, host_row, width,
+                                  static_cast<size_t>(L), cudaMemcpyHostToDevice,
+                                  hp->in) != cudaSuccess)
                 return cuda_fail();
         if (cudaEventRecord(hp->in_done[slot], hp->in) != cudaSuccess ||
-            cudaStreamWaitEvent(st, hp->in_done[slot], 0) != cudaSuccess)
+            cudaStreamWaitEvent(cs, hp->in_done[slot], 0) != cudaSuccess)
             return cuda_fail();
-        // forward and backward of sample z on the caller's stream
-        s = fwd_impl(base, base + per, base + 2 * per, base + 4 * per, lens, lens + 1, 1, L, L, H, D,
-                     alpha, bias, nullptr, dtype, stream);
+        // forward and backward of the unit, as one sample of hc heads
+        s = fwd_impl(base, base + slot_tensor, base + 2 * slot_tensor, base + 4 * slot_tensor, lens,
+                     lens + 1, 1, L, L, hc, D, alpha, bias, nullptr, dtype, cs);
         if (s != SIGATTN_OK) return s;
-        s = bwd_impl(base, base + per, base + 2 * per, base + 3 * per, base + 5 * per,
-                     base + 6 * per, base + 7 * per, lens, lens + 1, 1, L, L, H, D, alpha, bias,
-                     dtype, stream, kPartDq | kPartDkdv);
+        s = bwd_impl(base, base + slot_tensor, base + 2 * slot_tensor, base + 3 * slot_tensor,
+                     base + 5 * slot_tensor, base + 6 * slot_tensor, base + 7 * slot_tensor, lens,
+                     lens + 1, 1, L, L, hc, D, alpha, bias, dtype, cs, kPartDq | kPartDkdv);
         if (s != SIGATTN_OK) return s;
-        if (cudaEventRecord(hp->comp_done[slot], st) != cudaSuccess ||
+        if (cudaEventRecord(hp->comp_done[slot], cs) != cudaSuccess ||
             cudaStreamWaitEvent(hp->out, hp->comp_done[slot], 0) != cudaSuccess)
             return cuda_fail();
-        // outputs of sample z back to the host while the next sample computes
+        // outputs back to their rows of the host tensors while later units compute
         for (int t = 0; t < 4; ++t)
-            if (cudaMemcpyAsync(static_cast<uint8_t *>(hout[t]) + z * per, base + (4 + t) * per, per,
-                                cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+            if (cudaMemcpy2DAsync(hout[t] + host_off, host_row, base + (4 + t) * slot_tensor, width,
+                                  width, static_cast<size_t>(L), cudaMemcpyDeviceToHost,
+                                  hp->out) != cudaSuccess)
                 return cuda_fail();
         if (cudaEventRecord(hp->freed[slot], hp->out) != cudaSuccess) return cuda_fail();
     }
-    // the call completes on `stream` once every output has reached the host
-    for (int slot = 0; slot < (Z > 1 ? 2 : 1); ++slot)
-        if (cudaStreamWaitEvent(st, hp->freed[slot], 0) != cudaSuccess) return cuda_fail();
+    // the call completes on `stream` once every output has reached the host (the
+    // copy-out stream runs in unit order, so its last event covers all units)
+    if (cudaStreamWaitEvent(st, hp->freed[(units - 1) % kPipeSlots], 0) != cudaSuccess)
+        return cuda_fail();
     return SIGATTN_OK;
 }
 
