@@ -139,8 +139,9 @@ sigattn_status sigattn_bwd_rect(const void *q, const void *k, const void *v, con
 
 /* Forward and backward of a batch held in HOST memory, with the transfers
  * overlapped.  The batch is cut into units of one sample and a group of heads
- * (whole samples once Z >= 8; otherwise about 8 units in all, so that the
- * first copy in and the last copy out, which nothing overlaps, are short).
+ * (about 16 units in all, so that the first copy in and the last copy out,
+ * which nothing overlaps, are short, but never less than 8 MB per tensor of a
+ * unit, so that whole samples stay whole when they are small).
  * Per unit, its rows of q, k, v, dout (host, [Z][L][H][D]) are copied into a
  * compact device slot on a library-owned copy stream while earlier units
  * compute; the forward and the backward of the unit run on one of two

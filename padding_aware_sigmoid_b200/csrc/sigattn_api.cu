@@ -59,12 +59,21 @@ struct HostPipe {
                 freed[kPipeSlots] = {};
 };
 
-// The pipeline's unit of work: `hc` heads (the last unit of a sample may have
-// fewer) of one sample.  A batch of few samples is split by heads so that the
-// first copy in and the last copy out, which nothing overlaps, are short.
-constexpr int kPipeUnitsTarget = 8;
-int pipe_heads_per_unit(int Z, int H) {
-    const int chunks = std::min(H, (kPipeUnitsTarget + Z - 1) / Z);
+// The pipeline's unit of work: a group of heads of one sample (the last group
+// of a sample may be smaller).  A batch of few samples is split by heads into
+// about kPipeUnitsTarget units, so that the first copy in and the last copy
+// out, which nothing overlaps, are short; but one tensor of a unit keeps at
+// least kPipeMinUnitBytes, below which the kernels' launches are too small to
+// fill the GPU.  The groups are made as even as the head count allows.
+constexpr int kPipeUnitsTarget = 16;
+constexpr size_t kPipeMinUnitBytes = size_t(8) << 20;
+int pipe_heads_per_unit(int Z, int L, int H, int D, size_t elem_bytes) {
+    int chunks = std::min(H, (kPipeUnitsTarget + Z - 1) / Z);
+    int hpu = (H + chunks - 1) / chunks;
+    const size_t per_head = static_cast<size_t>(L) * D * elem_bytes;
+    const size_t min_heads = (kPipeMinUnitBytes + per_head - 1) / per_head;
+    hpu = std::max(hpu, static_cast<int>(std::min<size_t>(H, min_heads)));
+    chunks = (H + hpu - 1) / hpu;
     return (H + chunks - 1) / chunks;
 }
 HostPipe g_pipe[kMaxDevices];
@@ -437,8 +446,8 @@ sigattn_status sigattn_bwd_rect(const void *q, const void *k, const void *v, con
 size_t sigattn_fwd_bwd_host_workspace_bytes(int Z, int L, int H, int D, sigattn_dtype dtype) {
     if (Z <= 0 || L <= 0 || H <= 0 || (D != 64 && D != 128)) return 0;
     if (dtype != SIGATTN_BF16 && dtype != SIGATTN_FP32) return 0;
-    const size_t per = static_cast<size_t>(L) * pipe_heads_per_unit(Z, H) * D *
-                       (dtype == SIGATTN_BF16 ? 2 : 4);
+    const size_t es = dtype == SIGATTN_BF16 ? 2 : 4;
+    const size_t per = static_cast<size_t>(L) * pipe_heads_per_unit(Z, L, H, D, es) * D * es;
     // kPipeSlots unit slots of eight tensors, then one 256-byte length record per slot
     return kPipeSlots * 8 * per + kPipeSlots * 256;
 }
@@ -469,7 +478,7 @@ sigattn_status sigattn_fwd_bwd_host(const void *q, const void *k, const void *v,
     if ((s = host_pipe(dev, &hp)) != SIGATTN_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t es = dtype == SIGATTN_BF16 ? 2 : 4;
-    const int hpu = pipe_heads_per_unit(Z, H);
+    const int hpu = pipe_heads_per_unit(Z, L, H, D, es);
     const int chunks = (H + hpu - 1) / hpu;
     const size_t slot_tensor = static_cast<size_t>(L) * hpu * D * es;   // one tensor of a slot
     const size_t host_row = static_cast<size_t>(H) * D * es;             // one row of a host tensor
