@@ -136,7 +136,12 @@ def _check(code: int, where: str):
 
 
 def _stream_ptr(t) -> int:
+    """Raw handle of the current stream on t's device (what torch.cuda.current_stream
+    returns, without building a Stream object on every call)."""
     import torch
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return raw(t.get_device())
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
@@ -152,18 +157,19 @@ def _dtype_code(t) -> int:
 def _check_inputs(tensors, seqlens):
     import torch
     ref = tensors[0]
-    if ref.dim() != 4:
+    shape, dtype, device = ref.shape, ref.dtype, ref.device
+    if len(shape) != 4:
         raise ValueError("tensors must be [Z, L, H, D]")
+    if not ref.is_cuda:
+        raise ValueError("sigattn tensors must live on a CUDA device (no CPU fallback)")
     for t in tensors:
-        if not t.is_cuda:
-            raise ValueError("sigattn tensors must live on a CUDA device (no CPU fallback)")
-        if t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+        if t is not ref and (t.shape != shape or t.dtype != dtype or t.device != device):
             raise ValueError("all tensors must share shape, dtype and device")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous [Z, L, H, D]")
     for s in seqlens:
-        if not (s.is_cuda and s.dtype == torch.int32 and s.dim() == 1 and s.shape[0] == ref.shape[0]
-                and s.is_contiguous() and s.device == ref.device):
+        if not (s.device == device and s.dtype == torch.int32 and s.dim() == 1
+                and s.shape[0] == shape[0] and s.is_contiguous()):
             raise ValueError("seqlens must be contiguous int32 [Z] tensors on the tensors' device")
 
 
