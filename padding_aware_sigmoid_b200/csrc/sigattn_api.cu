@@ -8,6 +8,8 @@
 #include <atomic>
 #include <cstdio>
 #include <mutex>
+#include <unordered_map>
+#include <unordered_set>
 
 #include "../../include/sigattn.h"
 #include "bwd_sm100.cuh"
@@ -143,7 +145,8 @@ sigattn_status get_encoder() {
 
 // [Z][L][H][D] bf16 viewed as a 4-D tensor (D, H, L, Z), boxes of 64 x 1 x 128 x 1
 // elements with 128-byte swizzle: one box is one [128 rows][64 cols] operand atom.
-sigattn_status encode_bf16_map(CUtensorMap *m, const void *base, int Z, int L, int H, int D) {
+sigattn_status encode_bf16_map_uncached(CUtensorMap *m, const void *base, int Z, int L, int H,
+                                        int D) {
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                           static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(Z)};
     cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
@@ -158,6 +161,46 @@ sigattn_status encode_bf16_map(CUtensorMap *m, const void *base, int Z, int L, i
         g_last_cuda_error.store(10000 + static_cast<int>(r));
         return SIGATTN_ERR_CUDA;
     }
+    return SIGATTN_OK;
+}
+
+// Encoded maps, keyed by everything that goes into one: a bf16 map is a pure
+// function of (base address, Z, L, H, D), so a hit returns exactly what a new
+// encoding would, and repeated calls on the same buffers skip the driver call.
+// Bounded: the cache is emptied when it reaches kMaxCachedMaps entries.
+struct MapKey {
+    const void *base;
+    int Z, L, H, D;
+    bool operator==(const MapKey &o) const {
+        return base == o.base && Z == o.Z && L == o.L && H == o.H && D == o.D;
+    }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey &k) const {
+        size_t h = std::hash<const void *>()(k.base);
+        for (int v : {k.Z, k.L, k.H, k.D}) h = h * 1000003u ^ static_cast<size_t>(v);
+        return h;
+    }
+};
+constexpr size_t kMaxCachedMaps = 1024;
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
+
+sigattn_status encode_bf16_map(CUtensorMap *m, const void *base, int Z, int L, int H, int D) {
+    const MapKey key{base, Z, L, H, D};
+    {
+        std::lock_guard<std::mutex> lk(g_map_mu);
+        auto it = g_maps.find(key);
+        if (it != g_maps.end()) {
+            *m = it->second;
+            return SIGATTN_OK;
+        }
+    }
+    sigattn_status s = encode_bf16_map_uncached(m, base, Z, L, H, D);
+    if (s != SIGATTN_OK) return s;
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    if (g_maps.size() >= kMaxCachedMaps) g_maps.clear();
+    g_maps.emplace(key, *m);
     return SIGATTN_OK;
 }
 
@@ -189,13 +232,36 @@ sigattn_status check_lengths(int Z, int Lq, int Lk, int H, int D, sigattn_dtype 
     return (Lq == 0 || Lk == 0) ? SIGATTN_ERR_INVALID_ARG : SIGATTN_OK;
 }
 
+// (kernel, device) pairs whose dynamic shared-memory limit has been raised; a
+// kernel always asks for the same amount, so once per device is enough.
+struct FuncDev {
+    const void *f;
+    int dev;
+    bool operator==(const FuncDev &o) const { return f == o.f && dev == o.dev; }
+};
+struct FuncDevHash {
+    size_t operator()(const FuncDev &k) const {
+        return std::hash<const void *>()(k.f) * 31u ^ static_cast<size_t>(k.dev);
+    }
+};
+std::mutex g_attr_mu;
+std::unordered_set<FuncDev, FuncDevHash> g_attr_set;
+
 template <typename... KArgs, typename... Args>
 sigattn_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                       cudaStream_t stream, Args... args) {
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return cuda_fail(e);
+        const FuncDev key{reinterpret_cast<const void *>(kernel), dev};
+        std::lock_guard<std::mutex> lk(g_attr_mu);
+        if (g_attr_set.count(key) == 0) {
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem));
+            if (e != cudaSuccess) return cuda_fail(e);
+            g_attr_set.insert(key);
+        }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
