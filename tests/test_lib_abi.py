@@ -157,3 +157,32 @@ def test_launch_order_is_a_stable_descending_sort(lib):
     assert lib.sigattn_launch_order(None, 3, None) == 1
     assert lib.sigattn_launch_order(None, -1, None) == 1
     assert lib.sigattn_launch_order(None, 0, None) == 0
+
+
+def test_host_pipeline_units_from_workspace_size(lib):
+    """The host-buffer call cuts a batch into about 16 (sample, head group) units
+    of at least 8 MB per tensor, groups as even as the heads allow; its
+    workspace is three unit slots of eight tensors plus 256 bytes per slot, so
+    the size shows the heads per unit."""
+    import math
+    import torch
+    import padding_aware_sigmoid_b200 as sa
+
+    def heads_per_unit(Z, L, H, D, es):
+        chunks = min(H, -(-16 // Z))
+        hpu = -(-H // chunks)
+        per_head = L * D * es
+        hpu = max(hpu, min(H, -(-(8 << 20) // per_head)))
+        chunks = -(-H // hpu)
+        return -(-H // chunks)
+
+    cases = [((2, 16384, 16, 128), torch.bfloat16, 2), ((4, 16384, 16, 128), torch.bfloat16, 4),
+             ((8, 2048, 12, 64), torch.bfloat16, 12), ((4, 8192, 12, 64), torch.bfloat16, 6),
+             ((1, 16384, 5, 128), torch.bfloat16, 2), ((1, 8192, 4, 128), torch.float32, 2),
+             ((3, 384, 2, 128), torch.bfloat16, 2)]
+    for (Z, L, H, D), dt, want in cases:
+        es = 4 if dt == torch.float32 else 2
+        assert heads_per_unit(Z, L, H, D, es) == want
+        assert sa.fwd_bwd_host_workspace_bytes(Z, L, H, D, dt) == 3 * 8 * L * want * D * es + 3 * 256
+    assert lib.sigattn_fwd_bwd_host_workspace_bytes(0, 128, 1, 64, 0) == 0
+    assert lib.sigattn_fwd_bwd_host_workspace_bytes(1, 128, 1, 96, 0) == 0
