@@ -299,8 +299,7 @@ def e2e_workload(sa, w, steps, warmup, device):
     """Same step through the public API with host buffers: sigattn_fwd_bwd_host
     copies Q, K, V, dO from pinned host memory, runs the forward and the backward,
     and copies O, dQ, dK, dV back, unit by unit (a sample and a group of heads)
-    with the copies overlapping
-    the compute; all of it inside the timed region."""
+    with the copies overlapping the compute; all of it inside the timed region."""
     import torch
     from padding_aware_sigmoid_b200 import workloads as W
     hq, hk, hv, hdo = (torch.empty((w.Z, w.L, w.H, w.D), dtype=torch.bfloat16).pin_memory()
