@@ -27,8 +27,15 @@
  * device status word (see sigattn_last_device_status).
  *
  * Ownership: the caller owns and allocates every buffer; calls allocate
- * nothing per call.  The library lazily allocates, once per device, a small
- * device status buffer that lives until process exit.
+ * no device memory per call.  The library lazily allocates, once per device,
+ * a small device status buffer that lives until process exit.  In host
+ * memory it caches the TMA tensor maps it encodes, keyed by (base address,
+ * Z, L, H, D), which is all a map depends on (at most 1024, then the cache is
+ * emptied).
+ *
+ * CUDA graphs: the compute calls (not sigattn_fwd_bwd_host) can be captured
+ * after a first call on the device; a replay reads the lengths and tensors
+ * from the captured addresses again.
  *
  * Asynchrony: every compute call enqueues its kernels on `stream` (a
  * cudaStream_t passed as void*; NULL = the legacy default stream) and
