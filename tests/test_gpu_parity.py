@@ -291,3 +291,18 @@ def test_host_buffer_pipeline_matches_device_path(Z, L, H, D, dtype):
     ref = _run(inp, dev)
     for name, a, b in zip(("O", "dQ", "dK", "dV"), outs, ref):
         assert torch.equal(a, b.cpu()), name
+
+
+@pytest.mark.parametrize("Z", [40, 70])
+def test_many_samples_launch_order(Z):
+    """Up to 64 samples the kernels rank them by length with two samples per
+    lane (Z = 40 uses both); above 64 they keep the index order (Z = 70).  Lengths
+    are shuffled, with ties and empty samples; every output must still match."""
+    dev = _dev()
+    L, H, D = 256, 1, 64
+    g = np.random.default_rng(Z)
+    nq = g.integers(0, L + 1, size=Z)
+    nk = g.integers(0, L + 1, size=Z)
+    nq[::7], nk[::5], nk[3] = 0, L, nk[4]
+    inp = _case(Z, L, H, D, nq, nk, seed=8000 + Z)
+    _check_full(inp, _run(inp, dev), "bf16")
