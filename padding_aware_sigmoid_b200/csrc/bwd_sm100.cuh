@@ -71,6 +71,9 @@ struct BwdLayout {
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
+// ring depths per head dimension: X (dq: K, dkdv: Q) and Y (dq: V, dkdv: dO) slots
+template <int D> struct BwdStages { static constexpr int X = D == 128 ? 3 : 4, Y = D == 128 ? 2 : 4; };
+
 // Streams tiles j = 0..n-1 of one tensor map into a ring of S slots; returns
 // false when a wait gave up.  `issued` counts the loads issued so far.
 template <int S, int NSUB>

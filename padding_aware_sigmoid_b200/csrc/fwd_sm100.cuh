@@ -8,13 +8,19 @@
 // without any load (the pages' block-sparse skip, paperlayer.ai summary,
 // section 4).
 //
-// Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles once, then K_j into the key ring
-//   warp 2      TMA producer: V_j into the value ring
-//   warp 1      owns TMEM; one thread issues every tcgen05.mma
-//   warps 4-7   sigma warpgroup 0: keys [0,64) of each tile (thread = query row),
-//               then the epilogue of query tile 0
-//   warps 8-11  sigma warpgroup 1: keys [64,128) of each tile, epilogue of tile 1
+// Warp roles (640 threads):
+//   warp 0       TMA producer: Q tiles once, then K_j into the key ring
+//   warp 2       TMA producer: V_j into the value ring
+//   warp 1       owns TMEM; one thread issues every tcgen05.mma
+//   warp 3       idle
+//   warps 4-19   four sigma warpgroups (thread = query row = TMEM lane):
+//                warpgroup g serves query tile t = g / 2, key columns
+//                [64 c, 64 c + 64) of each key tile with c = g % 2, then
+//                writes columns [c D/2, c D/2 + D/2) of tile t's output.
+// Each SM sub-partition thus runs four sigma warps, two per query tile, so
+// one tile's sigma work keeps the MUFU busy while the other tile's warps wait
+// for their next scores (the MUFU reaches its full rate only with two or more
+// warps issuing on a sub-partition).
 // Tensor memory (512 columns, fp32):
 //   [0,128) S0   [128,256) S1   [256,256+D) O0   [256+D,256+2D) O1
 // P_t (bf16, two per column) overwrites S_t columns [0,32) (keys 0-63) and
@@ -87,8 +93,12 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, 
     }
 }
 
+constexpr int kFwdThreads = 640;
+// ring depths per head dimension: key slots K and value slots V
+template <int D> struct FwdStages { static constexpr int K = D == 128 ? 2 : 4, V = D == 128 ? 3 : 4; };
+
 template <int D, int MODE, int KS, int VS>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using Lay = FwdLayout<D, KS, VS>;
@@ -123,7 +133,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&s_full[t], 1);
-            mbar_init(&p_full[t], 256);  // both sigma warpgroups
+            mbar_init(&p_full[t], 256);  // the two sigma warpgroups of tile t
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -258,15 +268,16 @@ __global__ void __launch_bounds__(384, 1)
                 trace(1, j, 0);
                 for (int t = 0; t < ntiles; ++t) {
                     if (!(ok = mbar_wait(&p_full[t], j & 1, wctx))) break;
-                    trace(1, j, 1 + 2 * t);
+                    trace(1, j, 1 + 3 * t);
                     tc_fence_after();
                     issue_pv(t, vbase, j == 0);
+                    trace(1, j, 2 + 3 * t);
                     if (t == ntiles - 1) mma_commit(&v_empty[stv]);
                     if (more) {
                         if (t == 0 && !(ok = mbar_wait(&k_full[stk], ((j + 1) / KS) & 1, wctx))) break;
-                        trace(1, j, 2 + 2 * t);
                         tc_fence_after();
                         issue_s(t, knext);
+                        trace(1, j, 3 + 3 * t);
                         if (t == ntiles - 1) mma_commit(&k_empty[stk]);
                     }
                 }
@@ -277,75 +288,77 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ sigma warpgroups
-        // Both warpgroups work on every query tile, warpgroup g on key columns
-        // [64 g, 64 g + 64) of S_t, so each sigma phase has two warps per SM
-        // sub-partition: one warp per sub-partition cannot keep the MUFU busy
-        // (its dependent chain leaves issue slots empty).  The tiles alternate:
-        // while the warpgroups evaluate tile t, the tensor pipe runs the other
-        // tile's P.V and next scores.
+        // Warpgroup g works on query tile t = g / 2 only, on key columns
+        // [64 c, 64 c + 64) of S_t (c = g % 2).  The warpgroups of the two tiles
+        // run side by side on every SM sub-partition: while one tile's warps
+        // wait for their next scores (P.V and the next Q K^T of that tile on
+        // the tensor pipe), the other tile's warps keep the MUFU busy.
         const int g = (warp - 4) >> 2;
+        const int t = g >> 1, c = g & 1;
         const int quarter = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
         bool ok = true;
-        if (work) {
+        const bool mine = work && t < ntiles;
+        if (mine) {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
-            // one flat loop over (key tile j, query tile t) steps, t fastest
-            const int nsteps = nkv * ntiles;
-            for (int it = 0; it < nsteps; ++it) {
-                const int t = ntiles == 2 ? (it & 1) : 0;
-                const int j = ntiles == 2 ? (it >> 1) : it;
-                if (quarter == 0) trace(2 + g, j, 2 * t);
+            const uint32_t tS = tmem + lane_bits + (t ? Lay::COL_S1 : Lay::COL_S0) + 64 * c;
+            for (int j = 0; j < nkv; ++j) {
+                if (quarter == 0) trace(2 + c, j, 2 * t);
                 ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wctx));
                 if (!ok) break;
-                if (quarter == 0) trace(2 + g, j, 2 * t + 1);
+                if (quarter == 0) trace(2 + c, j, 2 * t + 1);
                 tc_fence_after();
-                const uint32_t tS = tmem + lane_bits + (t ? Lay::COL_S1 : Lay::COL_S0) + 64 * g;
-                uint32_t r[64];
-                tmem_ld64(tS, r);
-                uint32_t pk[32];
+                const int kvalid = nk - j * Lay::BN - 64 * c;  // keys of this half below n_k
+                // two chunks of 32 scores per thread; P of chunk u lies over S
+                // columns [16 u, 16 u + 16) of this half, already read
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float2 pr = sigma2<MODE>(
-                        scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
-                    pk[i] = pack_bf16x2(pr.x, pr.y);
-                }
-                const int kvalid = nk - j * Lay::BN - 64 * g;  // keys of this half below n_k
-                if (kvalid < 64) {
-                    // last key tile: keys at or beyond n_k weigh exactly zero
+                for (int u = 0; u < 2; ++u) {
+                    uint32_t r[32];
+                    tmem_ld32(tS + 32 * u, r);
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const uint32_t lo = 2 * i < kvalid ? 0x0000FFFFu : 0u;
-                        const uint32_t hi = 2 * i + 1 < kvalid ? 0xFFFF0000u : 0u;
-                        pk[i] &= (lo | hi);
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 pr = sigma2<MODE>(
+                            scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf));
+                        pk[i] = pack_bf16x2(pr.x, pr.y);
                     }
+                    if (kvalid < 64) {
+                        // last key tile: keys at or beyond n_k weigh exactly zero
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int col = 32 * u + 2 * i;
+                            const uint32_t lo = col < kvalid ? 0x0000FFFFu : 0u;
+                            const uint32_t hi = col + 1 < kvalid ? 0xFFFF0000u : 0u;
+                            pk[i] &= (lo | hi);
+                        }
+                    }
+                    tmem_st16(tS + 16 * u, pk);
                 }
-                // P of these 64 keys lies over the first 32 of the S columns
-                // just read; the other warpgroup never touches them
-                tmem_st32(tS, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[t]);
-                if (quarter == 0) trace(2 + g, j, 4 + t);
+                if (quarter == 0) trace(2 + c, j, 4 + t);
             }
             // every MMA of this CTA has finished once the MMA thread's final commit lands
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
         }
-        // epilogue: warpgroup g writes query tile g
-        const int row = (qtile0 + g) * Lay::BM + quarter * 32 + lane;
+        // epilogue: warpgroup g writes columns [c D/2, c D/2 + D/2) of query tile t
+        constexpr int HALF = D / 2;
+        const int row = (qtile0 + t) * Lay::BM + quarter * 32 + lane;
         const size_t row_stride = static_cast<size_t>(p.H) * D;
         __nv_bfloat16 *orow = p.o + (static_cast<size_t>(z) * L + row) * row_stride +
-                              static_cast<size_t>(h) * D;
-        if (work && g < ntiles) {
+                              static_cast<size_t>(h) * D + c * HALF;
+        if (mine) {
             if (ok) {
                 tc_fence_after();
-                const uint32_t tO = tmem + lane_bits + (g ? Lay::COL_O1 : Lay::COL_O0);
+                const uint32_t tO = tmem + lane_bits + (t ? Lay::COL_O1 : Lay::COL_O0) + c * HALF;
                 const bool valid = row < nq;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int cc = 0; cc < HALF / 32; ++cc) {
                     uint32_t r[32];
-                    tmem_ld32(tO + 32 * c, r);
+                    tmem_ld32(tO + 32 * cc, r);
                     if (row < L) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * cc);
 #pragma unroll
                         for (int v4 = 0; v4 < 4; ++v4) {
                             uint4 w;
@@ -362,7 +375,7 @@ __global__ void __launch_bounds__(384, 1)
             // query tile wholly in padding, or no valid key: exact zeros, no loads
             uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-            for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+            for (int v4 = 0; v4 < HALF / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
 
