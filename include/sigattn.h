@@ -211,6 +211,14 @@ sigattn_status sigattn_bwd_bias(const void *q, const void *k, const void *v, con
                                 const int32_t *seqlens_k, int Z, int L, int H, int D, float alpha,
                                 const float *bias, float *dbias, void *workspace,
                                 size_t workspace_bytes, sigattn_dtype dtype, void *stream);
+/* The pages' per-sample bias b_z = -ln n_z (paperlayer.ai summary, section 3;
+ * gist.science summary, section 2.A), for sigattn_fwd_bias / sigattn_bwd_bias:
+ * seqlens is a device int32[Z] (typically seqlens_k), bias a device float[Z]
+ * that receives -logf(n_z), or 0 where n_z <= 1.  Asynchronous on `stream`.
+ * Errors: SIGATTN_ERR_INVALID_ARG for Z < 0 or a NULL pointer with Z > 0,
+ * SIGATTN_ERR_CUDA for a launch failure. */
+sigattn_status sigattn_log_length_bias(const int32_t *seqlens, int Z, float *bias, void *stream);
+
 /* Bytes of device workspace sigattn_bwd_bias needs to return dbias (0 for an
  * empty problem): one float per dQ work unit (bf16: per 128-row query tile
  * and head; fp32: per query row and head) of every sample. */
@@ -248,11 +256,12 @@ sigattn_status sigattn_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
 /* Forward for callers that must not allocate device memory.
  *
  * No counterpart in the paper; this is a deployment convenience.  Some
- * callers cannot call cudaMalloc at the time they run attention: code
- * running inside a CUDA-graph capture, inside a framework whose caching
- * allocator owns all device memory, or in a service that reserves its memory
- * at start-up and forbids allocation on the request path.  Such callers
- * often also have the per-sample lengths only on the host.  This entry point
+ * callers cannot call cudaMalloc at the time they run attention: code running
+ * inside a framework whose caching allocator owns all device memory (a
+ * cudaMalloc behind its back can fail or fragment the pool it manages), or a
+ * service that reserves its memory at start-up and forbids allocation on the
+ * request path (an allocation there can stall or fail under load).  Such
+ * callers often also have the per-sample lengths only on the host.  This entry point
  * computes exactly what sigattn_fwd computes, with the same kernel, but takes
  * seqlens_q / seqlens_k as HOST int32[Z] arrays and never allocates: the
  * lengths and the kernel's device status word live in a fixed array in the
@@ -263,8 +272,10 @@ sigattn_status sigattn_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
  *  - Z <= SIGATTN_NOALLOC_MAX_Z (8192), else SIGATTN_ERR_TOO_LARGE and
  *    nothing is launched.  Lengths are checked on the host: any value
  *    outside [0, L] returns SIGATTN_ERR_SEQLEN_RANGE before any launch.
- *  - The host arrays may be reused as soon as the call returns (they are
- *    staged with cudaMemcpyAsync from pageable memory).
+ *  - The host arrays are read during the call: their values reach the
+ *    device as kernel arguments (up to 480 samples per small launch), so
+ *    they may be reused or freed as soon as the call returns, pageable or
+ *    pinned alike.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress); make that first call before any stream capture.
  *  - Every call shares the one array, and it keeps the last call's contents

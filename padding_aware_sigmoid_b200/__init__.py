@@ -23,7 +23,7 @@ __all__ = [
     "version", "library_path", "load_library", "SIGMOID_TANH", "SIGMOID_EXP", "EXPORTS",
     "SigmoidAttention", "bwd_dq", "bwd_dkdv", "last_cuda_error", "fwd_noalloc", "NOALLOC_MAX_Z",
     "fwd_bias", "bwd_bias", "dbias_workspace_bytes", "fwd_rect", "bwd_rect", "fwd_bwd_host",
-    "fwd_bwd_host_workspace_bytes", "launch_order",
+    "fwd_bwd_host_workspace_bytes", "launch_order", "log_length_bias",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -52,7 +52,7 @@ EXPORTS = (
     "sigattn_last_cuda_error", "sigattn_status_string", "sigattn_version",
     "sigattn_fwd_noalloc", "sigattn_fwd_bias", "sigattn_bwd_bias", "sigattn_dbias_workspace_bytes",
     "sigattn_fwd_rect", "sigattn_bwd_rect", "sigattn_fwd_bwd_host",
-    "sigattn_fwd_bwd_host_workspace_bytes", "sigattn_launch_order",
+    "sigattn_fwd_bwd_host_workspace_bytes", "sigattn_launch_order", "sigattn_log_length_bias",
 )
 
 
@@ -123,6 +123,8 @@ def load_library():
         lib.sigattn_status_string.argtypes = [ci]
         lib.sigattn_status_string.restype = ctypes.c_char_p
         lib.sigattn_version.restype = ci
+        lib.sigattn_log_length_bias.argtypes = [vp, ci, vp, vp]
+        lib.sigattn_log_length_bias.restype = ci
         lib.sigattn_launch_order.argtypes = [vp, ci, vp]
         lib.sigattn_launch_order.restype = ci
         _lib = lib
@@ -357,6 +359,21 @@ def fwd_bias(q, k, v, seqlens_q, seqlens_k, alpha: float, bias, out=None):
     return out
 
 
+def log_length_bias(seqlens):
+    """b_z = -ln n_z (0 where n_z <= 1) as a float32 [Z] tensor on the lengths'
+    device, computed by the library: the pages' per-sample bias for ``fwd_bias``
+    and ``bwd_bias``.  ``seqlens``: int32 [Z] CUDA tensor."""
+    import torch
+    if not (seqlens.is_cuda and seqlens.dtype == torch.int32 and seqlens.is_contiguous()
+            and seqlens.dim() == 1):
+        raise ValueError("seqlens must be a contiguous int32 [Z] CUDA tensor")
+    out = torch.empty(seqlens.shape, dtype=torch.float32, device=seqlens.device)
+    _check(load_library().sigattn_log_length_bias(seqlens.data_ptr(), int(seqlens.numel()),
+                                                  out.data_ptr(), _stream_ptr(seqlens)),
+           "sigattn_log_length_bias")
+    return out
+
+
 def dbias_workspace_bytes(Z: int, L: int, H: int, dtype) -> int:
     """Device workspace bytes ``bwd_bias`` needs to return the bias gradient."""
     import torch
@@ -406,10 +423,11 @@ def fwd_noalloc(q, k, v, seqlens_q, seqlens_k, alpha: float, bias: float, out=No
         out = torch.empty_like(q)
     else:
         _check_inputs([q, out], [])
-    nq = np.ascontiguousarray(np.asarray(seqlens_q.cpu() if hasattr(seqlens_q, "cpu") else seqlens_q,
-                                         dtype=np.int32).reshape(-1))
-    nk = np.ascontiguousarray(np.asarray(seqlens_k.cpu() if hasattr(seqlens_k, "cpu") else seqlens_k,
-                                         dtype=np.int32).reshape(-1))
+    # private copies: the call reads them on the host before it returns
+    nq = np.array(seqlens_q.cpu() if hasattr(seqlens_q, "cpu") else seqlens_q,
+                  dtype=np.int32, copy=True).reshape(-1)
+    nk = np.array(seqlens_k.cpu() if hasattr(seqlens_k, "cpu") else seqlens_k,
+                  dtype=np.int32, copy=True).reshape(-1)
     Z, L, H, D = (int(s) for s in q.shape)
     if nq.shape[0] != Z or nk.shape[0] != Z:
         raise ValueError("seqlens must have Z entries")

@@ -58,12 +58,17 @@ class SigmoidAttention(torch.nn.Module):
     (paperlayer.ai summary, section 3; gist.science summary, section 2.A):
 
     * default: one scalar, ``bias`` or -ln(L) with n the padded length;
-    * ``per_sample_bias=True``: b_z = -ln n_k(z), each sample's true length;
-    * ``learnable_bias=True``: a scalar parameter (initial value ``bias`` or
-      -ln(L) of the first batch) trained through db = sum_z db_z."""
+    * ``per_sample_bias=True``: b_z = -ln n_k(z), each sample's true length
+      (computed on the device by the library, ``log_length_bias``);
+    * ``learnable_bias=True``: a scalar parameter trained through
+      db = sum_z db_z, created here with the initial value ``bias``, or -ln
+      ``max_len`` (the padded length the module will see) when ``bias`` is not
+      given, so that an optimiser built from ``parameters()`` before the first
+      call already holds it."""
 
     def __init__(self, alpha: float | None = None, bias: float | None = None,
-                 per_sample_bias: bool = False, learnable_bias: bool = False):
+                 per_sample_bias: bool = False, learnable_bias: bool = False,
+                 max_len: int | None = None):
         super().__init__()
         if per_sample_bias and learnable_bias:
             raise ValueError("choose per_sample_bias or learnable_bias, not both")
@@ -71,8 +76,12 @@ class SigmoidAttention(torch.nn.Module):
         self.per_sample_bias = per_sample_bias
         self.learnable_bias = learnable_bias
         self.b = None
-        if learnable_bias and bias is not None:
-            self.b = torch.nn.Parameter(torch.tensor(float(bias)))
+        if learnable_bias:
+            if bias is None and max_len is None:
+                raise ValueError("learnable_bias needs an initial value: give bias, or max_len "
+                                 "for b = -ln(max_len)")
+            init = float(bias) if bias is not None else -math.log(max_len)
+            self.b = torch.nn.Parameter(torch.tensor(init))
 
     def forward(self, q, k, v, seqlens_q, seqlens_k=None):
         if seqlens_k is None:
@@ -80,11 +89,10 @@ class SigmoidAttention(torch.nn.Module):
         Z, L, D = q.shape[0], q.shape[1], q.shape[-1]
         alpha = float(1.0 / math.sqrt(D) if self.alpha is None else self.alpha)
         if self.per_sample_bias:
-            bias_z = -torch.log(seqlens_k.to(torch.float32).clamp(min=1.0))
+            from . import log_length_bias
+            bias_z = log_length_bias(seqlens_k)
             return _SigmoidAttentionBiasFn.apply(q, k, v, seqlens_q, seqlens_k, alpha, bias_z)
         if self.learnable_bias:
-            if self.b is None:
-                self.b = torch.nn.Parameter(torch.tensor(-math.log(L), device=q.device))
             bias_z = self.b.to(device=q.device, dtype=torch.float32).expand(Z)
             return _SigmoidAttentionBiasFn.apply(q, k, v, seqlens_q, seqlens_k, alpha, bias_z)
         bias = -math.log(L) if self.bias is None else self.bias

@@ -21,10 +21,6 @@ namespace {
 using namespace sigattn;
 
 constexpr int kMaxDevices = 64;
-// forward rings: key and value slots per head dim
-template <int D> struct FwdStages { static constexpr int K = D == 128 ? 2 : 4, V = D == 128 ? 3 : 4; };
-// backward rings: X (dq: K, dkdv: Q) and Y (dq: V, dkdv: dO) slots per head dim
-template <int D> struct BwdStages { static constexpr int X = D == 128 ? 3 : 4, Y = D == 128 ? 2 : 4; };
 
 std::mutex g_mu;
 int *g_status[kMaxDevices] = {};          // device status word per device (lazy, never freed)
@@ -41,7 +37,13 @@ sigattn_status cuda_fail(cudaError_t e = cudaSuccess) {
     return SIGATTN_ERR_CUDA;
 }
 
-// Current device, its compute capability and its status word.
+// b_z = -ln n_z for each sample; 0 for n_z <= 1 (a sample with no key has
+// nothing to weigh, and one key gives ln 1 = 0).
+__global__ void log_length_bias_kernel(const int32_t *n, int Z, float *bias) {
+    const int z = blockIdx.x * blockDim.x + threadIdx.x;
+    if (z < Z) bias[z] = n[z] > 1 ? -logf(static_cast<float>(n[z])) : 0.0f;
+}
+
 // Writes one sample's two lengths into device memory; the values travel as
 // kernel arguments, so nothing is read from host memory after the call returns.
 __global__ void store_lengths_kernel(int32_t *dst, int32_t nq, int32_t nk) {
@@ -278,7 +280,7 @@ sigattn_status fwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
                         const FwdParams &p, int Z, int L, int H, cudaStream_t st) {
     constexpr int KS = FwdStages<D>::K, VS = FwdStages<D>::V;
     dim3 grid((L + 255) / 256, H, Z);
-    return launch(fwd_kernel<D, MODE, KS, VS>, grid, dim3(384), FwdLayout<D, KS, VS>::SMEM_ALLOC, st,
+    return launch(fwd_kernel<D, MODE, KS, VS>, grid, dim3(kFwdThreads), FwdLayout<D, KS, VS>::SMEM_ALLOC, st,
                   mq, mk, mv, p);
 }
 
@@ -608,6 +610,13 @@ sigattn_status sigattn_fwd_bwd_host(const void *q, const void *k, const void *v,
     return SIGATTN_OK;
 }
 
+sigattn_status sigattn_log_length_bias(const int32_t *seqlens, int Z, float *bias, void *stream) {
+    if (Z < 0 || (Z > 0 && (!seqlens || !bias))) return SIGATTN_ERR_INVALID_ARG;
+    if (Z == 0) return SIGATTN_OK;
+    return launch(log_length_bias_kernel, dim3((Z + 255) / 256), dim3(256), 0,
+                  static_cast<cudaStream_t>(stream), seqlens, Z, bias);
+}
+
 sigattn_status sigattn_set_sigmoid_mode(sigattn_sigmoid_mode mode) {
     if (mode != SIGATTN_SIGMOID_TANH && mode != SIGATTN_SIGMOID_EXP) return SIGATTN_ERR_INVALID_ARG;
     g_sigmoid_mode.store(mode == SIGATTN_SIGMOID_TANH ? kSigmoidTanh : kSigmoidExp);
@@ -723,6 +732,25 @@ sigattn_status noalloc_scratch(int dev, int32_t **ptr) {
     *ptr = g_noalloc_ptr[dev];
     return SIGATTN_OK;
 }
+
+// The lengths reach the array as kernel arguments, in chunks that keep one
+// launch's parameters under 4 KB, so nothing is read from host memory after the
+// call returns, whatever kind of host memory holds them.  The chunk at z0 = 0
+// also clears the status word left by the previous call.
+constexpr int kLenChunk = 480;
+struct LenChunk {
+    int32_t nq[kLenChunk], nk[kLenChunk];
+    int z0, count;
+};
+static_assert(sizeof(LenChunk) <= 4000, "kernel parameter size");
+__global__ void store_length_chunk_kernel(int32_t *status, int32_t *nq, int32_t *nk,
+                                          const LenChunk c) {
+    for (int i = threadIdx.x; i < c.count; i += blockDim.x) {
+        nq[c.z0 + i] = c.nq[i];
+        nk[c.z0 + i] = c.nk[i];
+    }
+    if (c.z0 == 0 && threadIdx.x == 0) *status = 0;
+}
 }  // namespace
 
 extern "C" {
@@ -760,13 +788,20 @@ sigattn_status sigattn_fwd_noalloc(const void *q, const void *k, const void *v, 
     int32_t *nq = scratch + kNoallocHeader;
     int32_t *nk = scratch + kNoallocHeader + SIGATTN_NOALLOC_MAX_Z;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // the array keeps the previous call's contents: clear the status word
-    if ((e = cudaMemsetAsync(status, 0, sizeof(int32_t), st)) != cudaSuccess) return cuda_fail(e);
-    if ((e = cudaMemcpyAsync(nq, host_seqlens_q, sizeof(int32_t) * Z, cudaMemcpyHostToDevice, st)) !=
-            cudaSuccess ||
-        (e = cudaMemcpyAsync(nk, host_seqlens_k, sizeof(int32_t) * Z, cudaMemcpyHostToDevice, st)) !=
-            cudaSuccess)
-        return cuda_fail(e);
+    // the array keeps the previous call's contents: the first chunk clears the
+    // status word, and every length of this call is written before the forward
+    for (int z0 = 0; z0 < Z; z0 += kLenChunk) {
+        LenChunk c;
+        c.z0 = z0;
+        c.count = std::min(kLenChunk, Z - z0);
+        for (int i = 0; i < c.count; ++i) {
+            c.nq[i] = host_seqlens_q[z0 + i];
+            c.nk[i] = host_seqlens_k[z0 + i];
+        }
+        if ((s = launch(store_length_chunk_kernel, dim3(1), dim3(128), 0, st, status, nq, nk, c)) !=
+            SIGATTN_OK)
+            return s;
+    }
     if (dtype == SIGATTN_FP32) {
         F32Params p{static_cast<const float *>(q), static_cast<const float *>(k),
                     static_cast<const float *>(v), nullptr, static_cast<float *>(o), nullptr,

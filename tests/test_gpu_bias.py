@@ -270,3 +270,33 @@ def test_autograd_learnable_and_per_sample_bias():
     bz2 = (-np.log(nk.astype(np.float64))).astype(np.float32)
     C.assert_close(o2.float().cpu().numpy(), oracle.fwd(q, k, v, nq, nk, alpha, bz2), "bf16",
                    "O (per-sample -ln n)")
+
+
+def test_log_length_bias_matches_minus_ln_n():
+    """The library's b_z = -ln n_z, against numpy in fp64 rounded to fp32; n <= 1 gives 0."""
+    dev = _dev()
+    n = np.array([0, 1, 2, 3, 77, 128, 2048, 16384, 65536, 1 << 30], np.int32)
+    got = sa.log_length_bias(torch.as_tensor(n, device=dev)).cpu().numpy()
+    want = np.where(n > 1, -np.log(np.maximum(n, 1).astype(np.float64)), 0.0)
+    assert got.dtype == np.float32
+    assert np.all(np.abs(got - want) <= 2e-7 * np.maximum(np.abs(want), 1.0))
+    assert got[0] == 0.0 and got[1] == 0.0
+
+
+def test_learnable_bias_optimiser_built_before_first_call_updates_it():
+    """The learnable bias exists from construction, so an optimiser built before
+    the first call holds it and a step moves it by -lr * db."""
+    dev = _dev()
+    Z, L, H, D = 2, 256, 2, 64
+    q, k, v, do, nq, nk, _ = _inputs(Z, L, H, D, (256, 100), (256, 100), seed=3401)
+    mod = sa.SigmoidAttention(learnable_bias=True, max_len=L).to(dev)
+    assert abs(mod.b.item() + math.log(L)) < 1e-6
+    opt = torch.optim.SGD(mod.parameters(), lr=0.01)
+    b0 = mod.b.item()
+    o = mod(q.to(dev), k.to(dev), v.to(dev), torch.as_tensor(nq, device=dev),
+            torch.as_tensor(nk, device=dev))
+    o.backward(do.to(dev))
+    g = mod.b.grad.item()
+    opt.step()
+    assert g != 0.0
+    assert abs(mod.b.item() - (b0 - 0.01 * g)) <= 1e-6 * max(1.0, abs(b0))

@@ -1,15 +1,16 @@
 """The scratch-free forward (sigattn_fwd_noalloc) against the regular forward.
 
-Some callers cannot allocate device memory when they call attention (inside a
-CUDA-graph capture, under a framework allocator that owns the device memory, or
-in a service that reserves memory at start-up and forbids allocation later).
+Some callers cannot allocate device memory when they call attention: code
+inside a framework whose caching allocator owns the device memory, or a
+service that reserves its memory at start-up and forbids allocation later.
 For them the library offers a forward that keeps its scratch (the lengths and
 the kernel's status word) in a fixed array of its own device memory and takes
-the lengths on the host.  This test calls it through the C ABI twice in a row,
-with different inputs and lengths, and compares each result with the regular
-entry point's, within the bf16 parity tolerance the other tests use.  It lives
-in a file that pytest collects last, so a failure here never hides another
-test's result."""
+the lengths on the host.  Both entry points run the same kernel on the same
+data, so this test requires the results to be equal bit for bit, on two calls
+in a row with different shapes and lengths (the second call must not see the
+first one's lengths), and once more with the lengths in pinned host memory
+that is overwritten as soon as the call returns.  It lives in a file that
+pytest collects last, so a failure here never hides another test's result."""
 import math
 
 import numpy as np
@@ -49,13 +50,31 @@ def test_noalloc_forward_matches_regular_forward_twice():
         got = sa.fwd_noalloc(q, k, v, nq, nk, alpha, bias, out=out)
         torch.cuda.synchronize()
         assert got.data_ptr() == out.data_ptr()
-        g, r = got.float().cpu().numpy(), ref.float().cpu().numpy()
+        assert torch.equal(got, ref), "no-alloc forward differs from the regular forward"
+        g = got.float().cpu().numpy()
         for z in range(Z):
             assert np.all(g[z, nq[z]:] == 0.0), "padded query rows must be exactly zero"
-        if np.any(r != 0):
-            C.assert_close(g, r, "bf16", "O (no-alloc vs regular)")
-        else:
-            assert np.all(g == 0.0)
+
+
+def test_noalloc_forward_lengths_in_pinned_memory_reused_at_once():
+    dev = _dev()
+    Z, L, H, D = 600, 128, 1, 64     # more samples than one length launch carries
+    q, k, v = _inputs(Z, L, H, D, 3, dev)
+    n = np.random.default_rng(3).integers(0, L + 1, size=Z).astype(np.int32)
+    pq = torch.from_numpy(n.copy()).pin_memory()
+    pk = torch.from_numpy(n[::-1].copy()).pin_memory()
+    alpha, bias = 1.0 / math.sqrt(D), -math.log(L)
+    ref = sa.fwd(q, k, v, pq.to(dev), pk.to(dev), alpha, bias)
+    lib = sa.load_library()
+    out = torch.empty_like(q)
+    code = lib.sigattn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   pq.data_ptr(), pk.data_ptr(), Z, L, H, D, alpha, bias, 0,
+                                   torch.cuda.current_stream(dev).cuda_stream)
+    assert code == 0
+    pq.fill_(L)   # the call has returned: the library must not read these any more
+    pk.fill_(0)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
 
 
 def test_noalloc_forward_rejects_oversized_batch_and_bad_lengths():
