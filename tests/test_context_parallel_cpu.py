@@ -1,8 +1,10 @@
 """Context parallelism's exchange steps on CPU: world-size-2 gloo ranks each hold a
 slice of the sequence, all-gather K and V, compute their queries against every
-key and add the dK, dV contributions across ranks.  The per-rank compute is the
-fp64 oracle's rectangular route (the GPU kernels do not run on a CPU host); the
-reassembled result must equal the oracle on the unsplit sequence."""
+key and add the dK, dV contributions across ranks, both by the reduce-scatter
+on the chunked layout (the route NCCL takes) and by all-reduce and slice.  The
+per-rank compute is the fp64 oracle's rectangular route (the GPU kernels do not
+run on a CPU host); the reassembled result must equal the oracle on the
+unsplit sequence."""
 import os
 import socket
 
@@ -39,7 +41,7 @@ def _free_port():
     return p
 
 
-def _worker(rank, world, port, q, k, v, do, n, alpha, bias, out):
+def _worker(rank, world, port, q, k, v, do, n, alpha, bias, out, method):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -50,7 +52,7 @@ def _worker(rank, world, port, q, k, v, do, n, alpha, bias, out):
         loc = [torch.from_numpy(np.ascontiguousarray(a[:, sl])) for a in (q, k, v, do)]
         nt = torch.from_numpy(n)
         o = cp.forward(loc[0], loc[1], loc[2], nt, alpha, bias, kernels=_OracleKernels)
-        dq, dk, dv = cp.backward(*loc, nt, alpha, bias, kernels=_OracleKernels)
+        dq, dk, dv = cp.backward(*loc, nt, alpha, bias, kernels=_OracleKernels, method=method)
         out.put((rank, o.numpy(), dq.numpy(), dk.numpy(), dv.numpy()))
     finally:
         dist.destroy_process_group()
@@ -64,8 +66,17 @@ def test_local_lengths():
         cp.local_lengths(n, 0, 3, 16)
 
 
+def test_chunked_layout_round_trip():
+    x = torch.arange(2 * 8 * 3 * 4, dtype=torch.float32).reshape(2, 8, 3, 4)
+    xt = cp.rows_to_chunks(x)
+    for r, chunk in enumerate(xt.chunk(4)):
+        # chunk r of the first dimension holds rank r's rows of every sample
+        assert torch.equal(cp.chunks_to_rows(chunk), x[:, 2 * r:2 * r + 2])
+
+
 @pytest.mark.timeout(300)
-def test_two_gloo_ranks_context_parallel():
+@pytest.mark.parametrize("method", ["reduce_scatter", "all_reduce"])
+def test_two_gloo_ranks_context_parallel(method):
     g = np.random.default_rng(1)
     Z, L, H, D = 3, 16, 2, 8
     q, k, v, do = (g.standard_normal((Z, L, H, D)).astype(np.float32) for _ in range(4))
@@ -74,7 +85,8 @@ def test_two_gloo_ranks_context_parallel():
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q, k, v, do, n, alpha, bias, out))
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q, k, v, do, n, alpha, bias, out,
+                                               method))
              for r in range(2)]
     for p in procs:
         p.start()
