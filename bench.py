@@ -4,15 +4,22 @@
 One step = one forward (sigattn_fwd) and one backward (sigattn_bwd: dQ kernel
 + dK/dV kernel) over one batch of the 16K / head-dim-128 kernel-benchmark
 workload without padding (Z=2, H=16, L=16384, D=128, bf16; paperlayer.ai
-summary, section 4).  The 25%-padding workload (Z=4, L=16384, n ~ U[8192,
-16384]) is measured the same way and reported beside it, with the padding
-loss.  Throughput counts valid-token FLOPs: 4 D H sum n_q n_k forward and 2.5x
-that backward (paperlayer.ai summary, appendix A.2).
+summary, section 4).  The padded workloads (Z=4, L=16384) are measured the
+same way and reported beside it with their padding loss.  Throughput counts
+valid-token FLOPs: 4 D H sum n_q n_k forward and 2.5x that backward
+(paperlayer.ai summary, appendix A.2).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Under torchrun every rank runs its own batch (weak scaling; the path shards
-over independent (z, h) problems with no collective); the time is the max over
-ranks.  Prints one JSON line on rank 0.
+With --gpus N > 1 and no torchrun environment, the script starts N ranks
+itself under torch.distributed.run (127.0.0.1).  Every rank runs its own batch
+(weak scaling: the path shards over independent (z, h) problems with no
+collective); the time is the max over ranks.  Prints one JSON line on rank 0.
+
+Profiling helpers (no JSON line):
+  --only fwd|dq|dkdv|all --shape Z,H,L,D   launches of one kernel on full lengths
+  --write-traffic CSV...                    writes profiles/traffic.json from ncu
+                                            CSV logs of dram__bytes_read.sum and
+                                            dram__bytes_write.sum
 """
 from __future__ import annotations
 
@@ -20,6 +27,8 @@ import argparse
 import json
 import math
 import os
+import re
+import socket
 import statistics
 import subprocess
 import sys
@@ -35,6 +44,9 @@ METRIC = "fwd/bwd TFLOPS (valid tokens) at L=16K d=128, 0%/25% pad; % of B200 BF
 HEADLINE = 3      # 16K, no padding
 PADDED = 4        # 16K, 25% padding
 L2_BYTES = 126 * 1024 * 1024
+# four lengths evenly spaced over the 25%-padding workload's range [8192, 16384]:
+# their mean is 12288 = 75% of L = 16384, so exactly 25% of the tokens are padding
+EXACT25_LENGTHS = (8192, 10923, 13653, 16384)
 
 
 def parse():
@@ -49,6 +61,10 @@ def parse():
                     help="launch only this kernel (profiling runs; prints timings, no JSON line)")
     ap.add_argument("--shape", default="2,16,4096,128", help="Z,H,L,D for --only")
     ap.add_argument("--sigmoid-mode", choices=["exp", "tanh"], default=None)
+    ap.add_argument("--write-traffic", nargs="+", default=None, metavar="CSV",
+                    help="write profiles/traffic.json from ncu CSV logs (no GPU needed)")
+    ap.add_argument("--no-eager", action="store_true",
+                    help="skip the PyTorch-eager context measurement")
     return ap.parse_args()
 
 
@@ -121,19 +137,34 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(args) -> int:
+    """Runs this script as `args.gpus` ranks under torch.distributed.run (one
+    node, rendezvous on 127.0.0.1) and returns its exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.run(cmd, timeout=3600).returncode
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        import datetime
-        import torch
-        import torch.distributed as dist
+        print(f"bench rank {rank} of {world} (local {local}) ready", file=sys.stderr, flush=True)
         if args.impl == "ours":
+            import datetime
+            import torch
+            import torch.distributed as dist
             torch.cuda.set_device(local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        else:
-            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
     return world, rank, local
 
 
@@ -201,7 +232,7 @@ def reference_arm(args, world, rank):
     sample = (f"{rows} query rows (fwd + dQ) and {rows} key rows (dK, dV) per step, drawn from "
               f"the {w.name} workload (Z={w.Z}, H={w.H}, L={w.L}, D={w.D})")
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
@@ -217,10 +248,11 @@ def reference_arm(args, world, rank):
 # ---------------------------------------------------------------- our arm
 
 
-def make_device_inputs(w, device, seed_offset: int):
+def make_device_inputs(w, device, seed_offset: int, lengths=None):
+    """Seeded device inputs of workload `w` (lengths: the workload's own unless given)."""
     import torch
     from padding_aware_sigmoid_b200 import workloads as W
-    n = W.lengths(w)
+    n = W.lengths(w) if lengths is None else np.asarray(lengths, np.int32)
     g = torch.Generator(device=device).manual_seed(1000 * w.index + seed_offset)
     q, k, v, do = (torch.randn((w.Z, w.L, w.H, w.D), generator=g, device=device,
                                dtype=torch.float32).mul_(w.qkv_scale if i < 3 else 1.0)
@@ -329,6 +361,60 @@ def e2e_workload(sa, w, steps, warmup, device):
     return ms, h2d, d2h
 
 
+def eager_sigmoid_attention(q, k, v, n, alpha: float, bias: float):
+    """Sigmoid attention written with plain PyTorch ops (the pages' PyTorch
+    baseline, paper.rainbus.top results table): the full score matrix is
+    materialised in bf16, masked by multiplication, then multiplied by V."""
+    import torch
+    Z, L, H, D = q.shape
+    qh, kh, vh = (t.permute(0, 2, 1, 3) for t in (q, k, v))
+    s = torch.matmul(qh, kh.transpose(-1, -2)) * alpha + bias
+    pos = torch.arange(L, device=q.device)
+    keep = (pos[None, :] < n[:, None]).to(q.dtype)            # [Z, L]
+    p = torch.sigmoid(s) * keep[:, None, None, :]
+    o = torch.matmul(p, vh) * keep[:, None, :, None]
+    return o.permute(0, 2, 1, 3)
+
+
+def eager_context(w, device, heads: int = 4, reps: int = 3):
+    """Context only, not the product: forward and backward of the PyTorch-eager
+    version on `heads` heads of one sample of workload `w` (its whole score
+    matrix fits in HBM), timed with CUDA events, in valid-FLOP TFLOPS."""
+    import torch
+    g = torch.Generator(device=device).manual_seed(11)
+    shape = (1, w.L, heads, w.D)
+    q, k, v, do = (torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
+                   for _ in range(4))
+    for t in (q, k, v):
+        t.requires_grad_(True)
+    n = torch.full((1,), w.L, dtype=torch.int32, device=device)
+    fl = 4.0 * w.D * heads * float(w.L) * w.L
+    st = torch.cuda.current_stream(device)
+    fwd, bwd = [], []
+    for i in range(reps + 1):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(st)
+        o = eager_sigmoid_attention(q, k, v, n, w.alpha, w.bias)
+        e[1].record(st)
+        o.backward(do)
+        e[2].record(st)
+        torch.cuda.synchronize(device)
+        if i > 0:
+            fwd.append(e[0].elapsed_time(e[1]))
+            bwd.append(e[1].elapsed_time(e[2]))
+        del o
+        q.grad = k.grad = v.grad = None
+    f_ms, b_ms = statistics.median(fwd), statistics.median(bwd)
+    del q, k, v, do
+    torch.cuda.empty_cache()
+    return {"fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tflops": fl / (f_ms * 1e-3) / 1e12,
+            "bwd_tflops": 2.5 * fl / (b_ms * 1e-3) / 1e12,
+            "slice": f"Z=1, H={heads}, L={w.L}, D={w.D}, full lengths, bf16 (a slice of the "
+                     f"{w.name} workload; every head costs the same)",
+            "note": "plain PyTorch ops with autograd on this GPU, timed as context for the "
+                    "pages' PyTorch rows; not part of the library"}
+
+
 def our_arm(args, world, rank, local):
     import torch
     import padding_aware_sigmoid_b200 as sa
@@ -339,7 +425,6 @@ def our_arm(args, world, rank, local):
     pk = peaks()
     w3, w4 = W.WORKLOADS[HEADLINE], W.WORKLOADS[PADDED]
     f3 = W.fwd_flops_valid(W.lengths(w3), W.lengths(w3), w3.H, w3.D)
-    f4 = W.fwd_flops_valid(W.lengths(w4), W.lengths(w4), w4.H, w4.D)
     f4_pad = W.fwd_flops_padded(w4.Z, w4.L, w4.H, w4.D)
 
     inp3 = make_device_inputs(w3, device, rank)
@@ -351,12 +436,34 @@ def our_arm(args, world, rank, local):
     step_ms = max_over_ranks(step_ms, world, device)
     barrier(world)
     del inp3
-    inp4 = make_device_inputs(w4, device, rank)
-    step4_ms, fwd4_ms, dq4_ms, dkdv4_ms = time_workload(sa, w4, inp4, max(args.steps // 2, 3),
-                                                         args.warmup, device)
-    step4_ms = max_over_ranks(step4_ms, world, device)
-    del inp4
-    torch.cuda.empty_cache()
+    # Padding: the 25%-padding workload as drawn (lengths U[8192, 16384] from its
+    # seed), the same Z = 4 shape with no padding (so that the loss compares like
+    # grids), and lengths evenly spaced over [8192, 16384] whose tokens are
+    # exactly 25% padding (mean fill 75%, as the workload intends).
+    pad_runs = {}
+    for name, lens in (("drawn", W.lengths(w4)), ("nopad_z4", [w4.L] * w4.Z),
+                       ("exact25", EXACT25_LENGTHS)):
+        inp4 = make_device_inputs(w4, device, rank, lengths=lens)
+        st_ms, f_ms, q_ms, kv_ms = time_workload(sa, w4, inp4, max(args.steps // 2, 3),
+                                                 args.warmup, device)
+        st_ms = max_over_ranks(st_ms, world, device)
+        fl = W.fwd_flops_valid(lens, lens, w4.H, w4.D)
+        pad_runs[name] = {
+            "lengths": [int(x) for x in lens],
+            "token_padding_fraction": 1.0 - float(np.sum(lens)) / (w4.Z * w4.L),
+            "valid_fraction_of_padded_flops": fl / f4_pad,
+            "fwd_ms": f_ms, "bwd_dq_ms": q_ms, "bwd_dkdv_ms": kv_ms, "ms_per_step": st_ms,
+            "fwd_tflops": fl / (f_ms * 1e-3) / 1e12,
+            "bwd_tflops": 2.5 * fl / ((q_ms + kv_ms) * 1e-3) / 1e12,
+            "fwd_tflops_padded_flops": f4_pad / (f_ms * 1e-3) / 1e12,
+        }
+        del inp4
+        torch.cuda.empty_cache()
+    ref = pad_runs["nopad_z4"]
+    for name in ("drawn", "exact25"):
+        r = pad_runs[name]
+        r["fwd_padding_loss_pct"] = 100.0 * (1.0 - r["fwd_tflops"] / ref["fwd_tflops"])
+        r["bwd_padding_loss_pct"] = 100.0 * (1.0 - r["bwd_tflops"] / ref["bwd_tflops"])
 
     # each kernel also timed on its own (10 back-to-back launches after the step
     # loop): the GPU's power-limited clock then follows that kernel alone
@@ -424,6 +531,10 @@ def our_arm(args, world, rank, local):
         e2e = {"value": world * f3 * 3.5 / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    eager = None
+    if rank == 0 and not args.no_eager:
+        eager = eager_context(w3, device)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -442,8 +553,6 @@ def our_arm(args, world, rank, local):
     fwd_tf = f3 / (fwd_ms * 1e-3) / 1e12
     bwd_tf = 2.5 * f3 / ((dq_ms + dkdv_ms) * 1e-3) / 1e12
     step_tf = world * 3.5 * f3 / (step_ms * 1e-3) / 1e12
-    fwd4_tf = f4 / (fwd4_ms * 1e-3) / 1e12
-    bwd4_tf = 2.5 * f4 / ((dq4_ms + dkdv4_ms) * 1e-3) / 1e12
     # dominant kernel: the longest of the three per step
     kernels = {"fwd": (fwd_ms, f3), "bwd_dkdv": (dkdv_ms, 8.0 / 4.0 * f3),
                "bwd_dq": (dq_ms, 6.0 / 4.0 * f3)}
@@ -484,14 +593,13 @@ def our_arm(args, world, rank, local):
         },
         "fwd_pct_of_peak": 100.0 * fwd_tf / pk["bf16"],
         "bwd_pct_of_peak": 100.0 * bwd_tf / pk["bf16"],
-        "pad25": {
-            "workload": w4.name, "lengths": [int(x) for x in W.lengths(w4)],
-            "fwd_tflops": fwd4_tf, "bwd_tflops": bwd4_tf,
-            "fwd_tflops_padded_flops": f4_pad / (fwd4_ms * 1e-3) / 1e12,
-            "fwd_padding_loss_pct": 100.0 * (1.0 - fwd4_tf / fwd_tf),
-            "bwd_padding_loss_pct": 100.0 * (1.0 - bwd4_tf / bwd_tf),
-            "ms_per_step": step4_ms,
-        },
+        "pad25": dict(
+            pad_runs,
+            note="loss = 1 - valid-FLOP TFLOPS of the padded batch / that of the same Z = 4 "
+                 "shape without padding; 'drawn' is the workload's seeded draw, 'exact25' has "
+                 "exactly 25% padded tokens",
+            fwd_padding_loss_pct=pad_runs["exact25"]["fwd_padding_loss_pct"],
+            bwd_padding_loss_pct=pad_runs["exact25"]["bwd_padding_loss_pct"]),
         "workloads_d64": d64,
         "roofline": {
             "kernel": dom, "bound": "tensor", "achieved": achieved, "peak": pk["bf16"],
@@ -504,16 +612,27 @@ def our_arm(args, world, rank, local):
         "gpu_launches": 3 * args.steps,   # the timed headline steps: fwd, dQ, dK/dV
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "context": {"pytorch_eager": eager},
     }
     print(json.dumps(line), flush=True)
 
 
+# the device code: every file a kernel is compiled from, including the ring
+# depths and thread counts; host code (argument checks, caches, launches) is not
+# part of it
+DEVICE_SOURCES = ("fwd_sm100.cuh", "fwd_persist_sm100.cuh", "bwd_sm100.cuh", "sm100.cuh",
+                  "sigmoid.cuh")
+TRAFFIC_KERNELS = {"fwd": "fwd_tiles_kernel", "bwd_dq": "bwd_dq_kernel",
+                   "bwd_dkdv": "bwd_dkdv_kernel"}
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")
+
+
 def kernel_source_hash() -> str:
-    """sha256 over the CUDA sources of the library (file names and contents)."""
+    """sha256 over the device-code headers of the library (names and contents)."""
     import hashlib
     h = hashlib.sha256()
     src = os.path.join(ROOT, "padding_aware_sigmoid_b200", "csrc")
-    for name in sorted(os.listdir(src)):
+    for name in DEVICE_SOURCES:
         h.update(name.encode())
         with open(os.path.join(src, name), "rb") as f:
             h.update(f.read())
@@ -522,16 +641,72 @@ def kernel_source_hash() -> str:
 
 def _ncu_traffic(kernel: str):
     """DRAM bytes per launch from the committed ncu capture of the same kernel,
-    or None when there is none or the kernel sources changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    or None when there is none or the device code changed since it was taken."""
     try:
-        with open(path) as f:
+        with open(TRAFFIC_PATH) as f:
             d = json.load(f)
         if d.get("_meta", {}).get("source_sha256") != kernel_source_hash():
             return None
         return d.get(kernel)
     except Exception:
         return None
+
+
+_BYTE_UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12}
+
+
+def read_ncu_dram_csv(path: str) -> dict:
+    """Per kernel name: list of (read + write) DRAM bytes, one per captured launch,
+    from an `ncu --csv --log-file` of dram__bytes_read.sum and dram__bytes_write.sum."""
+    import csv
+    rows = []
+    with open(path, newline="") as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    for r in csv.DictReader(lines):
+        rows.append(r)
+    per_launch = {}
+    for r in rows:
+        m = r.get("Metric Name", "")
+        if m not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        unit = r.get("Metric Unit", "byte").strip().lower()
+        val = float(r["Metric Value"].replace(",", "")) * _BYTE_UNITS[unit]
+        key = (r["ID"], r["Kernel Name"])
+        per_launch[key] = per_launch.get(key, 0.0) + val
+    out = {}
+    for (_, name), v in sorted(per_launch.items(), key=lambda kv: int(kv[0][0])):
+        out.setdefault(name, []).append(v)
+    return out
+
+
+def write_traffic(paths, command: str = "") -> dict:
+    """Writes profiles/traffic.json from ncu CSV logs: the mean bytes per launch of
+    each library kernel found, the algorithmic bytes of the workload the captures
+    ran on (workload 3 at full size), and the hash of the current device code."""
+    from padding_aware_sigmoid_b200 import workloads as W
+    w = W.WORKLOADS[HEADLINE]
+    tensor = w.Z * w.L * w.H * w.D * 2
+    got = {}
+    for p in paths:
+        for name, vals in read_ncu_dram_csv(p).items():
+            for key, kname in TRAFFIC_KERNELS.items():
+                if re.search(r"(^|[\s:])%s(<|\(|$)" % kname, name):
+                    got.setdefault(key, []).extend(vals)
+    d = {k: int(round(sum(v) / len(v))) for k, v in got.items()}
+    d["_meta"] = {
+        "what": "dram__bytes_read.sum + dram__bytes_write.sum per launch, mean over the "
+                "captured launches, workload %s (Z=%d, H=%d, L=%d, D=%d), full size" % (
+                    w.name, w.Z, w.H, w.L, w.D),
+        "launches": {k: len(v) for k, v in got.items()},
+        "algorithmic_bytes": {"fwd": 4 * tensor, "bwd_dq": 5 * tensor, "bwd_dkdv": 6 * tensor},
+        "source_sha256": kernel_source_hash(),
+        "device_sources": list(DEVICE_SOURCES),
+        "command": command,
+    }
+    with open(TRAFFIC_PATH, "w") as f:
+        json.dump(d, f, indent=1)
+        f.write("\n")
+    return d
 
 
 def only_kernel(args):
@@ -573,12 +748,17 @@ def only_kernel(args):
 
 def main():
     args = parse()
+    if args.write_traffic is not None:
+        print(json.dumps(write_traffic(args.write_traffic, os.environ.get("TRAFFIC_COMMAND", ""))))
+        return
     if args.sigmoid_mode is not None:
         import padding_aware_sigmoid_b200 as sa
         sa.set_sigmoid_mode(sa.SIGMOID_TANH if args.sigmoid_mode == "tanh" else sa.SIGMOID_EXP)
     if args.only is not None:
         only_kernel(args)
         return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args))
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
@@ -586,7 +766,7 @@ def main():
         else:
             our_arm(args, world, rank, local)
     finally:
-        if world > 1:
+        if world > 1 and args.impl == "ours":
             import torch.distributed as dist
             dist.destroy_process_group()
 

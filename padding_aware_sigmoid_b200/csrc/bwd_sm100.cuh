@@ -21,7 +21,6 @@
 // while the warpgroups still work on the current tile.
 #pragma once
 
-#include "fwd_sm100.cuh"
 #include "sm100.cuh"
 #include "sigmoid.cuh"
 
@@ -121,10 +120,18 @@ __device__ __forceinline__ void store_row_from_tmem(uint32_t taddr, __nv_bfloat1
     }
 }
 
+// Zeroes rows [r0, r0 + rows) of head h of sample z in a [Z][L][H][D] bf16
+// tensor, 16 bytes per thread and step, with every thread of the block.
 template <int D>
-__device__ __forceinline__ void zero_row(__nv_bfloat16 *dst, int col0, int ncols) {
-    uint4 *o = reinterpret_cast<uint4 *>(dst + col0);
-    for (int v4 = 0; v4 < ncols / 8; ++v4) o[v4] = make_uint4(0u, 0u, 0u, 0u);
+__device__ __forceinline__ void zero_rows(__nv_bfloat16 *base, int z, int h, int r0, int rows, int L,
+                                          int H) {
+    constexpr int V4 = D / 8;   // 16-byte chunks per row
+    const size_t row_stride = static_cast<size_t>(H) * D;
+    for (int e = threadIdx.x; e < rows * V4; e += blockDim.x) {
+        uint4 *dst = reinterpret_cast<uint4 *>(base + (static_cast<size_t>(z) * L + r0 + e / V4) * row_stride +
+                                               static_cast<size_t>(h) * D);
+        dst[e % V4] = make_uint4(0u, 0u, 0u, 0u);
+    }
 }
 
 // Packs 32 pairs to bf16 and zeroes the entries at tile columns >= valid
@@ -185,6 +192,27 @@ __global__ void __launch_bounds__(384, 1)
     // samples start by decreasing key length: warp 0 picks this block's sample
     BlockSample *sample_slot = reinterpret_cast<BlockSample *>(smem + Lay::OFF_SAMPLE);
     if (warp == 0) publish_block_sample(p.seqlens_q, p.seqlens_k, true, sample_slot);
+    __syncthreads();
+    const BlockSample bs = *sample_slot;
+    const int z = bs.z, h = blockIdx.y, qtile = blockIdx.x;
+    const int L = p.Lq;     // rows of this kernel's tiles and outputs: queries
+    int nq = bs.nq, nk = bs.nk;
+    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
+        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
+        nq = min(max(nq, 0), L);
+        nk = min(max(nk, 0), p.Lk);
+    }
+    const int nkv = (nk + 127) / 128;
+    if (qtile * 128 >= nq || nkv == 0) {
+        // No valid (query, key) pair in this query tile: its dQ rows are zeros
+        // (and so is its share of db), written by every thread; the block ends
+        // here, before it sets up barriers or tensor memory.
+        zero_rows<D>(p.dq, z, h, qtile * 128, min(128, L - qtile * 128), L, p.H);
+        if constexpr (DB) {
+            if (threadIdx.x == 0) p.db_part[(static_cast<size_t>(z) * p.H + h) * gridDim.x + qtile] = 0.0f;
+        }
+        return;
+    }
     if (threadIdx.x == 0) {
         mbar_init(res_full, 1);
         for (int s = 0; s < SX; ++s) {
@@ -222,20 +250,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
 
-    const BlockSample bs = *sample_slot;
-    const int z = bs.z, h = blockIdx.y, qtile = blockIdx.x;
-    const int L = p.Lq;     // rows of this kernel's tiles and outputs: queries
-    int nq = bs.nq, nk = bs.nk;
-    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
-        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
-        nq = min(max(nq, 0), L);
-        nk = min(max(nk, 0), p.Lk);
-    }
-    const int nkv = (nk + 127) / 128;
-    const bool work = qtile * 128 < nq && nkv > 0;
 
     if (warp == 0) {
-        if (work && lane == 0) {
+        if (lane == 0) {
             uint8_t *sQ = smem + Lay::OFF_A, *sDO = smem + Lay::OFF_B;
             mbar_arrive_expect_tx(res_full, 2 * Lay::TILE_BYTES);
             for (int s = 0; s < Lay::NSUB; ++s) {
@@ -254,7 +271,7 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp == 2) {
         // V_j ring, fed by its own thread so it never waits behind a key slot
-        if (work && lane == 0) {
+        if (lane == 0) {
             int iy = 0;
             for (int j = 0; j < nkv; ++j) {
                 if (!ring_load<SY, Lay::NSUB>(&tmV, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
@@ -266,7 +283,7 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp == 1) {
         // the whole warp runs converged; elect.sync picks the issuing lane
-        if (work) {
+        {
             auto wait = [&](uint64_t *bar, uint32_t parity) {
                 return __all_sync(0xffffffffu, mbar_wait(bar, parity, wctx));
             };
@@ -337,7 +354,7 @@ __global__ void __launch_bounds__(384, 1)
                               static_cast<size_t>(h) * D;
         bool ok = true;
         float dbacc = 0.0f;   // bias gradient: sum of this row's dS (valid rows and keys)
-        if (work) {
+        {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             for (int j = 0; j < nkv; ++j) {
                 float2 g[32];
@@ -396,8 +413,6 @@ __global__ void __launch_bounds__(384, 1)
                 store_row_from_tmem<D>(tmem + lane_bits + kColDQ, drow, row < L, row < nq,
                                        p.alpha, w * (D / 2), D / 2);
             }
-        } else if (row < L) {
-            zero_row<D>(drow, w * (D / 2), D / 2);
         }
         if constexpr (DB) {
             // one partial per CTA, summed in a fixed order: warp sums, then the
@@ -416,9 +431,11 @@ __global__ void __launch_bounds__(384, 1)
         }
     }
 
+    // every warp converges before the block-wide barrier (the producer roles
+    // ran on one lane)
+    __syncwarp();
     __syncthreads();
     if (warp == 1) {
-        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, Lay::TMEM_COLS);
     }
@@ -470,6 +487,25 @@ __global__ void __launch_bounds__(384, 1)
     // samples start by decreasing query length: warp 0 picks this block's sample
     BlockSample *sample_slot = reinterpret_cast<BlockSample *>(smem + Lay::OFF_SAMPLE);
     if (warp == 0) publish_block_sample(p.seqlens_q, p.seqlens_k, false, sample_slot);
+    __syncthreads();
+    const BlockSample bs = *sample_slot;
+    const int z = bs.z, h = blockIdx.y, ktile = blockIdx.x;
+    const int L = p.Lk;     // rows of this kernel's tiles and outputs: keys
+    int nq = bs.nq, nk = bs.nk;
+    if (nq < 0 || nq > p.Lq || nk < 0 || nk > L) {
+        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
+        nq = min(max(nq, 0), p.Lq);
+        nk = min(max(nk, 0), L);
+    }
+    const int nqt = (nq + 127) / 128;
+    if (ktile * 128 >= nk || nqt == 0) {
+        // No valid (query, key) pair for this key tile: its dK and dV rows are
+        // zeros, written by every thread; the block ends here.
+        const int rows = min(128, L - ktile * 128);
+        zero_rows<D>(p.dk, z, h, ktile * 128, rows, L, p.H);
+        zero_rows<D>(p.dv, z, h, ktile * 128, rows, L, p.H);
+        return;
+    }
     if (threadIdx.x == 0) {
         mbar_init(res_full, 1);
         for (int s = 0; s < SX; ++s) {
@@ -505,20 +541,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
 
-    const BlockSample bs = *sample_slot;
-    const int z = bs.z, h = blockIdx.y, ktile = blockIdx.x;
-    const int L = p.Lk;     // rows of this kernel's tiles and outputs: keys
-    int nq = bs.nq, nk = bs.nk;
-    if (nq < 0 || nq > p.Lq || nk < 0 || nk > L) {
-        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
-        nq = min(max(nq, 0), p.Lq);
-        nk = min(max(nk, 0), L);
-    }
-    const int nqt = (nq + 127) / 128;
-    const bool work = ktile * 128 < nk && nqt > 0;
-
     if (warp == 0) {
-        if (work && lane == 0) {
+        if (lane == 0) {
             uint8_t *sK = smem + Lay::OFF_A, *sV = smem + Lay::OFF_B;
             mbar_arrive_expect_tx(res_full, 2 * Lay::TILE_BYTES);
             for (int s = 0; s < Lay::NSUB; ++s) {
@@ -538,7 +562,7 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp == 2) {
         // dO_i ring, fed by its own thread so it never waits behind a query slot
-        if (work && lane == 0) {
+        if (lane == 0) {
             int iy = 0;
             for (int i = 0; i < nqt; ++i) {
                 if (!ring_load<SY, Lay::NSUB>(&tmDO, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
@@ -551,7 +575,7 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp == 1) {
         // the whole warp runs converged; elect.sync picks the issuing lane
-        if (work) {
+        {
             auto wait = [&](uint64_t *bar, uint32_t parity) {
                 return __all_sync(0xffffffffu, mbar_wait(bar, parity, wctx));
             };
@@ -629,7 +653,7 @@ __global__ void __launch_bounds__(384, 1)
                             static_cast<size_t>(h) * D;
         __nv_bfloat16 *dst = (w == 0 ? p.dv : p.dk) + roff;
         bool ok = true;
-        if (work) {
+        {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             const uint32_t tS = tmem + lane_bits + Lay::COL_S + 64 * w;
             const uint32_t tD = tmem + lane_bits + Lay::COL_DP + 64 * w;
@@ -701,14 +725,14 @@ __global__ void __launch_bounds__(384, 1)
                 store_row_from_tmem<D>(tmem + lane_bits + (w == 0 ? Lay::COL_ACC0 : Lay::COL_ACC1), dst,
                                        row < L, row < nk, w == 0 ? 1.0f : p.alpha, 0, D);
             }
-        } else if (row < L) {
-            zero_row<D>(dst, 0, D);
         }
     }
 
+    // every warp converges before the block-wide barrier (the producer roles
+    // ran on one lane)
+    __syncwarp();
     __syncthreads();
     if (warp == 1) {
-        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, Lay::TMEM_COLS);
     }

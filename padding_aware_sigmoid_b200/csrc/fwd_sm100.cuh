@@ -1,12 +1,14 @@
-// Forward kernel: O = sigma(alpha Q K^T + b) V with key padding masked and
-// padded query rows zeroed (gist.science summary, section 2.A;
-// paper.rainbus.top summary, method steps (1)-(3)).
+// Forward kernel, one CTA per pair of query tiles (used for head dimension
+// 128): O = sigma(alpha Q K^T + b) V with key padding masked and padded query
+// rows zeroed (gist.science summary, section 2.A; paper.rainbus.top summary,
+// method steps (1)-(3)).  The persistent kernel for head dimension 64 is in
+// fwd_persist_sm100.cuh.
 //
 // One CTA owns two 128-row query tiles of one (z, h) and streams the key/value
 // tiles j < ceil(n_k / 128) through shared memory; key tiles wholly in padding
-// are never loaded, query tiles wholly in padding are written as zeros
-// without any load (the pages' block-sparse skip, paperlayer.ai summary,
-// section 4).
+// are never loaded.  A CTA whose tiles hold no valid (query, key) pair writes
+// its output rows as zeros and exits before it sets up barriers or tensor
+// memory (the pages' block-sparse skip, paperlayer.ai summary, section 4).
 //
 // Warp roles (640 threads):
 //   warp 0       TMA producer: Q tiles once, then K_j into the key ring
@@ -43,7 +45,7 @@ struct FwdParams {
     __nv_bfloat16 *o;
     const int *seqlens_q;
     const int *seqlens_k;
-    int Lq, Lk, H;          // padded lengths of Q (and O) and of K, V; heads
+    int Z, Lq, Lk, H;       // batch; padded lengths of Q (and O) and of K, V; heads
     float alpha, bias;
     int *status;
     uint64_t timeout_ns;
@@ -78,28 +80,13 @@ struct FwdLayout {
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ uint8_t *align_1k(uint8_t *p) {
-    uint32_t a = smem_u32(p);
-    return p + ((1024u - (a & 1023u)) & 1023u);
-}
-
-// Waits that never consult the abort flag: used to drain in-flight async work
-// before the CTA releases its shared and tensor memory.
-__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return;
-    uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > limit_ns) return;
-    }
-}
-
 constexpr int kFwdThreads = 640;
 // ring depths per head dimension: key slots K and value slots V
 template <int D> struct FwdStages { static constexpr int K = D == 128 ? 2 : 4, V = D == 128 ? 3 : 4; };
 
 template <int D, int MODE, int KS, int VS>
 __global__ void __launch_bounds__(kFwdThreads, 1)
-    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    fwd_tiles_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
     using Lay = FwdLayout<D, KS, VS>;
     extern __shared__ uint8_t smem_raw[];
@@ -121,6 +108,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // samples start by decreasing key length: warp 0 picks this block's sample
     BlockSample *sample_slot = reinterpret_cast<BlockSample *>(smem + Lay::OFF_SAMPLE);
     if (warp == 0) publish_block_sample(p.seqlens_q, p.seqlens_k, true, sample_slot);
+    __syncthreads();
+    const BlockSample bs = *sample_slot;
+    const int z = bs.z, h = blockIdx.y;
+    const int qtile0 = blockIdx.x * 2;
+    const int L = p.Lq;     // query rows of this problem (O has the same layout)
+    int nq = bs.nq, nk = bs.nk;
+    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
+        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
+        nq = min(max(nq, 0), L);
+        nk = min(max(nk, 0), p.Lk);
+    }
+    const int ntiles = (qtile0 * Lay::BM < nq ? 1 : 0) + ((qtile0 + 1) * Lay::BM < nq ? 1 : 0);
+    const int nkv = (nk + Lay::BN - 1) / Lay::BN;
+    const size_t row_stride = static_cast<size_t>(p.H) * D;
+    if (ntiles == 0 || nkv == 0) {
+        // No valid (query, key) pair in this block's tiles: its output rows are
+        // zeros, written by every thread, and the block ends here.
+        const int r0 = qtile0 * Lay::BM, rows = min(2 * Lay::BM, L - r0);
+        constexpr int V4 = D / 8;   // 16-byte chunks per row
+        for (int e = threadIdx.x; e < rows * V4; e += kFwdThreads) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(z) * L + r0 + e / V4) *
+                                                             row_stride + static_cast<size_t>(h) * D);
+            dst[e % V4] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        return;
+    }
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < KS; ++s) {
@@ -154,23 +167,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wctx{abort_flag, p.status, p.timeout_ns};
 
-    const BlockSample bs = *sample_slot;
-    const int z = bs.z, h = blockIdx.y;
-    const int qtile0 = blockIdx.x * 2;
-    const int L = p.Lq;     // query rows of this problem (O has the same layout)
-    int nq = bs.nq, nk = bs.nk;
-    if (nq < 0 || nq > L || nk < 0 || nk > p.Lk) {
-        if (threadIdx.x == 0) record_status(p.status, kStatusSeqlenRange);
-        nq = min(max(nq, 0), L);
-        nk = min(max(nk, 0), p.Lk);
-    }
-    const int ntiles = (qtile0 * Lay::BM < nq ? 1 : 0) + ((qtile0 + 1) * Lay::BM < nq ? 1 : 0);
-    const int nkv = (nk + Lay::BN - 1) / Lay::BN;
-    const bool work = ntiles > 0 && nkv > 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (work && lane == 0) {
+        if (lane == 0) {
             uint8_t *sQ = smem + Lay::OFF_Q;
             uint8_t *sK = smem + Lay::OFF_K;
             uint8_t *sV = smem + Lay::OFF_V;
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // ------------------------------------------------------------ value producer
         // V_j is released later than K_j, so its ring is fed by its own thread
         // and never waits behind a key slot.
-        if (work && lane == 0) {
+        if (lane == 0) {
             uint8_t *sV = smem + Lay::OFF_V;
             int issued_v = 0;
             for (int j = 0; j < nkv; ++j) {
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (work && lane == 0) {
+        if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(128, Lay::BN, false, false);
             const uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
             const uint32_t sQ = smem_u32(smem + Lay::OFF_Q);
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int quarter = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
         bool ok = true;
-        const bool mine = work && t < ntiles;
+        const bool mine = t < ntiles;
         if (mine) {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             const uint32_t tS = tmem + lane_bits + (t ? Lay::COL_S1 : Lay::COL_S0) + 64 * c;
@@ -345,7 +345,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // epilogue: warpgroup g writes columns [c D/2, c D/2 + D/2) of query tile t
         constexpr int HALF = D / 2;
         const int row = (qtile0 + t) * Lay::BM + quarter * 32 + lane;
-        const size_t row_stride = static_cast<size_t>(p.H) * D;
         __nv_bfloat16 *orow = p.o + (static_cast<size_t>(z) * L + row) * row_stride +
                               static_cast<size_t>(h) * D + c * HALF;
         if (mine) {
@@ -372,16 +371,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
             }
         } else if (row < L) {
-            // query tile wholly in padding, or no valid key: exact zeros, no loads
+            // the block's second query tile lies wholly in padding: exact zeros, no loads
             uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
             for (int v4 = 0; v4 < HALF / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
 
+    // every warp converges before the block-wide barrier (the producer and MMA
+    // roles ran on one lane)
+    __syncwarp();
     __syncthreads();
     if (warp == 1) {
-        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, Lay::TMEM_COLS);
     }

@@ -14,6 +14,7 @@
 #include "../../include/sigattn.h"
 #include "bwd_sm100.cuh"
 #include "fp32_simt.cuh"
+#include "fwd_persist_sm100.cuh"
 #include "fwd_sm100.cuh"
 
 namespace {
@@ -25,6 +26,7 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int *g_status[kMaxDevices] = {};          // device status word per device (lazy, never freed)
 int g_cc_major[kMaxDevices] = {};         // 0 = not queried yet
+int g_sm_count[kMaxDevices] = {};         // multiprocessors per device (persistent grids)
 std::atomic<int> g_sigmoid_mode{kSigmoidTanh};
 std::atomic<uint64_t> g_timeout_ns{4000000000ull};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -120,6 +122,10 @@ sigattn_status device_state(int *dev, int *cc_major, int **status) {
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess)
             return cuda_fail();
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
+            return cuda_fail();
+        g_sm_count[*dev] = sms;
         g_cc_major[*dev] = major * 10 + minor;
     }
     if (g_status[*dev] == nullptr) {
@@ -275,13 +281,27 @@ sigattn_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
     return SIGATTN_OK;
 }
 
+// Head dimension 128: one CTA per pair of query tiles (fwd_sm100.cuh).  Head
+// dimension 64: one CTA per SM, or per work item when there are fewer, each
+// walking its share of the items (fwd_persist_sm100.cuh).  At 64 the sigma
+// work dominates the short, ragged batches of the pages' workloads, where
+// block start-up, blocks over padded tiles and the last wave cost more than
+// the persistent loop's bookkeeping; at 128 the long sequences run faster
+// as independent blocks.
 template <int D, int MODE>
 sigattn_status fwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                        const FwdParams &p, int Z, int L, int H, cudaStream_t st) {
-    constexpr int KS = FwdStages<D>::K, VS = FwdStages<D>::V;
-    dim3 grid((L + 255) / 256, H, Z);
-    return launch(fwd_kernel<D, MODE, KS, VS>, grid, dim3(kFwdThreads), FwdLayout<D, KS, VS>::SMEM_ALLOC, st,
-                  mq, mk, mv, p);
+                        const FwdParams &p, int sms, cudaStream_t st) {
+    if constexpr (D == 64) {
+        const int64_t items = static_cast<int64_t>(p.Z) * p.H * ((p.Lq + 255) / 256);
+        dim3 grid(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(sms, items))));
+        return launch(fwd_persistent_kernel<D, MODE>, grid, dim3(kFwdThreads),
+                      FwdPersistLayout<D>::SMEM_ALLOC, st, mq, mk, mv, p);
+    } else {
+        constexpr int KS = FwdStages<D>::K, VS = FwdStages<D>::V;
+        dim3 grid((p.Lq + 255) / 256, p.H, p.Z);
+        return launch(fwd_tiles_kernel<D, MODE, KS, VS>, grid, dim3(kFwdThreads),
+                      FwdLayout<D, KS, VS>::SMEM_ALLOC, st, mq, mk, mv, p);
+    }
 }
 
 enum BwdParts : int { kPartDq = 1, kPartDkdv = 2 };
@@ -420,14 +440,14 @@ sigattn_status fwd_impl(const void *q, const void *k, const void *v, void *o,
     if ((s = encode_bf16_map(&mq, q, Z, Lq, H, D)) != SIGATTN_OK) return s;
     if ((s = encode_bf16_map(&mk, k, Z, Lk, H, D)) != SIGATTN_OK) return s;
     if ((s = encode_bf16_map(&mv, v, Z, Lk, H, D)) != SIGATTN_OK) return s;
-    FwdParams p{static_cast<__nv_bfloat16 *>(o), seqlens_q, seqlens_k, Lq, Lk, H, alpha, bias,
+    FwdParams p{static_cast<__nv_bfloat16 *>(o), seqlens_q, seqlens_k, Z, Lq, Lk, H, alpha, bias,
                 status, g_timeout_ns.load(), bias_z};
-    const int mode = g_sigmoid_mode.load();
+    const int mode = g_sigmoid_mode.load(), sms = g_sm_count[dev];
     if (D == 128)
-        return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, Z, Lq, H, st)
-                                    : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, Z, Lq, H, st);
-    return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, Z, Lq, H, st)
-                                : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, Z, Lq, H, st);
+        return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, sms, st)
+                                    : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, sms, st);
+    return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, sms, st)
+                                : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, sms, st);
 }
 
 }  // namespace
@@ -777,9 +797,10 @@ sigattn_status sigattn_fwd_noalloc(const void *q, const void *k, const void *v, 
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= kMaxDevices) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
     if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(e);
-    int major = 0, minor = 0;
+    int major = 0, minor = 0, sms = 0;
     if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return cuda_fail(e);
     if (dtype == SIGATTN_BF16 && major * 10 + minor != 100) return SIGATTN_ERR_UNSUPPORTED_DEVICE;
     int32_t *scratch = nullptr;
@@ -816,14 +837,14 @@ sigattn_status sigattn_fwd_noalloc(const void *q, const void *k, const void *v, 
     if ((s = encode_bf16_map(&mq, q, Z, L, H, D)) != SIGATTN_OK) return s;
     if ((s = encode_bf16_map(&mk, k, Z, L, H, D)) != SIGATTN_OK) return s;
     if ((s = encode_bf16_map(&mv, v, Z, L, H, D)) != SIGATTN_OK) return s;
-    FwdParams p{static_cast<__nv_bfloat16 *>(o), nq, nk, L, L, H, alpha, bias, status,
+    FwdParams p{static_cast<__nv_bfloat16 *>(o), nq, nk, Z, L, L, H, alpha, bias, status,
                 g_timeout_ns.load(), nullptr};
     const int mode = g_sigmoid_mode.load();
     if (D == 128)
-        return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
-                                    : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
-    return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, Z, L, H, st)
-                                : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, Z, L, H, st);
+        return mode == kSigmoidTanh ? fwd_bf16<128, kSigmoidTanh>(mq, mk, mv, p, sms, st)
+                                    : fwd_bf16<128, kSigmoidExp>(mq, mk, mv, p, sms, st);
+    return mode == kSigmoidTanh ? fwd_bf16<64, kSigmoidTanh>(mq, mk, mv, p, sms, st)
+                                : fwd_bf16<64, kSigmoidExp>(mq, mk, mv, p, sms, st);
 }
 
 #ifdef SIGATTN_TRACE
@@ -837,6 +858,19 @@ int sigattn_trace_dump(unsigned long long *dst, int n) {
         return -3;
     static unsigned long long zeros[kTraceRoles * kTraceSteps * kTraceEvents];
     if (cudaMemcpyToSymbol(g_sigattn_trace, zeros, sizeof zeros) != cudaSuccess) return -4;
+    return total;
+}
+
+// Diagnostic build only: copies the per-CTA log of the last launch (start ns,
+// end ns, smid << 32 | work, unused per CTA) to host memory and clears it.
+int sigattn_cta_log_dump(unsigned long long *dst, int n) {
+    const int total = kCtaLogMax * 8;
+    if (dst == nullptr || n < total) return -1;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -2;
+    if (cudaMemcpyFromSymbol(dst, g_sigattn_cta_log, sizeof(unsigned long long) * total) != cudaSuccess)
+        return -3;
+    static unsigned long long zeros[kCtaLogMax * 8];
+    if (cudaMemcpyToSymbol(g_sigattn_cta_log, zeros, sizeof zeros) != cudaSuccess) return -4;
     return total;
 }
 #endif

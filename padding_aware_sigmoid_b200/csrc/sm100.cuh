@@ -100,6 +100,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     }
 }
 
+// Waits that never consult the abort flag: used to drain in-flight async work
+// before the CTA releases its shared and tensor memory.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return;
+    uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) return;
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
@@ -188,6 +198,41 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// The same two MMA forms with each 64-bit shared-memory descriptor given as
+// its low and high 32-bit halves (see smem_desc_sw128): issuing loops keep one
+// base low word per operand and add a constant per K step, instead of
+// rebuilding the descriptor for every instruction.
+__device__ __forceinline__ void mma_ss_lh(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 da, {%1, %3};\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(accumulate), "r"(idesc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_lh(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(accumulate), "r"(idesc)
+        : "memory");
+}
+// Halves of smem_desc_sw128(start, lbo, sbo): the low word holds start >> 4 in
+// bits [0,14) (shared addresses stay below 2^18, so adding the >> 4 offset of
+// a later K step never carries out of the field) and lbo >> 4 in [16,30).
+__device__ __forceinline__ uint32_t desc_lo(uint32_t start, uint32_t lbo) {
+    return ((start >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo) {
+    return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
 
 // Warp-converged forms: the whole warp executes them and elect.sync picks the
@@ -416,6 +461,13 @@ __device__ __forceinline__ void publish_block_sample(const int32_t *seqlens_q,
 }
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+// Start of the dynamic shared memory rounded up to 1 KiB (the alignment of
+// the 128-byte-swizzled operand tiles); every layout reserves 1 KiB of slack.
+__device__ __forceinline__ uint8_t *align_1k(uint8_t *p) {
+    uint32_t a = smem_u32(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
 }  // namespace sigattn
@@ -426,7 +478,7 @@ __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 // at each role's waits and hand-offs into g_sigattn_trace[role][step][event],
 // read back with sigattn_trace_dump().  The default build compiles it away.
 namespace sigattn {
-constexpr int kTraceRoles = 4, kTraceSteps = 256, kTraceEvents = 8;
+constexpr int kTraceRoles = 8, kTraceSteps = 256, kTraceEvents = 8;
 #ifdef SIGATTN_TRACE
 __device__ unsigned long long g_sigattn_trace[kTraceRoles * kTraceSteps * kTraceEvents];
 __device__ __forceinline__ bool trace_cta() {
@@ -436,7 +488,28 @@ __device__ __forceinline__ void trace(int role, int step, int ev) {
     if (trace_cta() && (threadIdx.x & 31) == 0 && step < kTraceSteps)
         g_sigattn_trace[(role * kTraceSteps + step) * kTraceEvents + ev] = clock64();
 }
+// per-CTA record of one launch: start and end (%globaltimer), SM id, work
+constexpr int kCtaLogMax = 1 << 16;
+__device__ unsigned long long g_sigattn_cta_log[kCtaLogMax * 8];
+__device__ __forceinline__ uint32_t smid() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cta_log(int slot, unsigned long long v) {
+    const unsigned long long id = blockIdx.x + static_cast<unsigned long long>(gridDim.x) *
+                                  (blockIdx.y + static_cast<unsigned long long>(gridDim.y) * blockIdx.z);
+    if (threadIdx.x == 0 && id < kCtaLogMax) g_sigattn_cta_log[id * 8 + slot] = v;
+}
+__device__ __forceinline__ void cta_log_any(int slot, unsigned long long v) {
+    const unsigned long long id = blockIdx.x + static_cast<unsigned long long>(gridDim.x) *
+                                  (blockIdx.y + static_cast<unsigned long long>(gridDim.y) * blockIdx.z);
+    if (id < kCtaLogMax) g_sigattn_cta_log[id * 8 + slot] = v;
+}
 #else
 __device__ __forceinline__ void trace(int, int, int) {}
+__device__ __forceinline__ void cta_log(int, unsigned long long) {}
+__device__ __forceinline__ void cta_log_any(int, unsigned long long) {}
+__device__ __forceinline__ uint32_t smid() { return 0; }
 #endif
 }  // namespace sigattn

@@ -50,3 +50,48 @@ def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(monkeypatch):
             assert stored[k] <= 1.05 * stored["_meta"]["algorithmic_bytes"][k]
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 64)
     assert bench._ncu_traffic("bwd_dkdv") is None
+
+
+def test_traffic_written_from_ncu_csv_carries_the_device_code_hash(tmp_path, monkeypatch):
+    csv = tmp_path / "fwd.csv"
+    header = ('"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream",'
+              '"Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit",'
+              '"Metric Value"\n')
+    rows = []
+    for i, (rd, wr) in enumerate(((400.0, 110.0), (402.0, 112.0))):
+        for m, u, v in (("dram__bytes_read.sum", "Mbyte", rd), ("dram__bytes_write.sum", "Mbyte", wr),
+                        ("gpu__time_duration.sum", "msecond", 3.1)):
+            rows.append(f'"{i}","1","python","h","void sigattn::fwd_tiles_kernel<128, 0, 2, 3>(CUtensorMap_st)",'
+                        f'"1","7","(640, 1, 1)","(64, 16, 2)","0","10.0","Command line profiler metrics",'
+                        f'"{m}","{u}","{v}"\n')
+    csv.write_text("==PROF== a line ncu prints before the table\n" + header + "".join(rows))
+    out = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_PATH", str(out))
+    d = bench.write_traffic([str(csv)], "cmd")
+    assert d["fwd"] == 512_000_000 and d["_meta"]["launches"] == {"fwd": 2}
+    assert d["_meta"]["source_sha256"] == bench.kernel_source_hash()
+    assert bench._ncu_traffic("fwd") == 512_000_000
+    assert bench._ncu_traffic("bwd_dkdv") is None
+    # any edit of a device-code header invalidates the counters
+    monkeypatch.setattr(bench, "DEVICE_SOURCES", bench.DEVICE_SOURCES[:-1])
+    assert bench._ncu_traffic("fwd") is None
+
+
+def test_gpus_2_starts_two_ranks_and_reports_them():
+    """`bench.py --gpus 2` outside torchrun starts two ranks itself; on the
+    reference arm rank 0 alone times the oracle and prints the line, and the
+    line counts both ranks."""
+    import subprocess
+    import sys
+    import oracle
+    oracle.build()
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    ready = [ln for ln in r.stderr.splitlines() if ln.startswith("bench rank ")]
+    assert sorted(ready) == ["bench rank 0 of 2 (local 0) ready", "bench rank 1 of 2 (local 1) ready"]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["impl"] == "reference" and d["value"] > 0

@@ -270,6 +270,28 @@ def test_long_sequence_sampled(D, mode):
           {k: ("%.2e/%.2e" % v) for k, v in rep.items()})
 
 
+def test_tanh_margin_at_32k():
+    """The tanh form's error grows with L (b = -ln L pushes the scores into the
+    left tail, where 0.5 + 0.5 tanh cancels).  At L = 32768, D = 128, with one
+    full and one ragged sample, sampled rows of every output must pass the bf16
+    bar in tanh mode; the test prints the margin left to the L1 bar."""
+    dev = _dev()
+    Z, L, H, D = 2, 32768, 1, 128
+    n = (32768, 20001)
+    inp = _case(Z, L, H, D, n, n, seed=4300)
+    old = sa.get_sigmoid_mode()
+    sa.set_sigmoid_mode(sa.SIGMOID_TANH)
+    try:
+        outs = _run(inp, dev)
+    finally:
+        sa.set_sigmoid_mode(old)
+    rep = _check_sampled(inp, outs, 12, seed=43)
+    worst = max(v[1] for v in rep.values())
+    print(f"L=32768 D=128 sigma tanh: max-abs/max|ref| / L1 rel:",
+          {k: ("%.2e/%.2e" % v) for k, v in rep.items()},
+          f"worst L1 {worst:.2e} = {100 * worst / C.BF16_L1_REL:.0f}% of the bar")
+
+
 @pytest.mark.parametrize("Z,L,H,D,dtype", [(3, 384, 2, 128, "bf16"), (4, 256, 2, 64, "bf16"),
                                            (3, 200, 1, 64, "fp32"),
                                            (9, 130, 2, 64, "bf16"),
