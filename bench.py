@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--only", choices=["fwd", "dq", "dkdv", "all"], default=None,
                     help="launch only this kernel (profiling runs; prints timings, no JSON line)")
     ap.add_argument("--shape", default="2,16,4096,128", help="Z,H,L,D for --only")
+    ap.add_argument("--workload", type=int, default=None,
+                    help="with --only: run on this workload's shape, lengths and inputs instead")
     ap.add_argument("--sigmoid-mode", choices=["exp", "tanh"], default=None)
     ap.add_argument("--write-traffic", nargs="+", default=None, metavar="CSV",
                     help="write profiles/traffic.json from ncu CSV logs (no GPU needed)")
@@ -710,17 +712,28 @@ def write_traffic(paths, command: str = "") -> dict:
 
 
 def only_kernel(args):
-    """Profiling helper: W warm-up and K timed launches of one kernel on a
-    Z,H,L,D problem with full lengths, bf16, alpha = 1/sqrt(D), b = -ln L."""
+    """Profiling helper: W warm-up and K timed launches of one kernel, either on a
+    Z,H,L,D problem with full lengths (bf16, alpha = 1/sqrt(D), b = -ln L) or on
+    one workload's shape, lengths and seeded inputs (--workload)."""
     import torch
     import padding_aware_sigmoid_b200 as sa
-    Z, H, L, D = (int(x) for x in args.shape.split(","))
+    from padding_aware_sigmoid_b200 import workloads as W
     dev = torch.device("cuda", 0)
-    g = torch.Generator(device=dev).manual_seed(0)
-    q, k, v, do = (torch.randn((Z, L, H, D), generator=g, device=dev).to(torch.bfloat16)
-                   for _ in range(4))
-    n = torch.full((Z,), L, dtype=torch.int32, device=dev)
-    alpha, bias = 1.0 / math.sqrt(D), -math.log(L)
+    if args.workload is not None:
+        w = W.WORKLOADS[args.workload]
+        inp = make_device_inputs(w, dev, 0)
+        q, k, v, do, n = inp["q"], inp["k"], inp["v"], inp["dout"], inp["nq"]
+        Z, H, L, D = w.Z, w.H, w.L, w.D
+        alpha, bias = w.alpha, w.bias
+        flops = W.fwd_flops_valid(inp["n"], inp["n"], H, D)
+    else:
+        Z, H, L, D = (int(x) for x in args.shape.split(","))
+        g = torch.Generator(device=dev).manual_seed(0)
+        q, k, v, do = (torch.randn((Z, L, H, D), generator=g, device=dev).to(torch.bfloat16)
+                       for _ in range(4))
+        n = torch.full((Z,), L, dtype=torch.int32, device=dev)
+        alpha, bias = 1.0 / math.sqrt(D), -math.log(L)
+        flops = 4.0 * D * H * Z * L * L
     o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
     calls = {
         "fwd": lambda: sa.fwd(q, k, v, n, n, alpha, bias, out=o),
@@ -728,7 +741,6 @@ def only_kernel(args):
         "dkdv": lambda: sa.bwd_dkdv(q, k, v, do, n, n, alpha, bias, dk=dk, dv=dv),
     }
     names = list(calls) if args.only == "all" else [args.only]
-    flops = 4.0 * D * H * Z * L * L
     per = {"fwd": flops, "dq": 1.5 * flops, "dkdv": 2.0 * flops}
     for name in names:
         for _ in range(args.warmup):
@@ -741,8 +753,9 @@ def only_kernel(args):
         e.record()
         torch.cuda.synchronize()
         ms = s.elapsed_time(e) / args.steps
-        print(json.dumps({"kernel": name, "shape": [Z, H, L, D], "ms": ms,
-                          "tflops_executed": per[name] / ms / 1e9}), flush=True)
+        print(json.dumps({"kernel": name, "shape": [Z, H, L, D], "workload": args.workload,
+                          "ms": ms, "tflops_executed_valid_pairs": per[name] / ms / 1e9}),
+              flush=True)
     assert sa.last_device_status() == 0
 
 

@@ -315,6 +315,22 @@ def test_host_buffer_pipeline_matches_device_path(Z, L, H, D, dtype):
         assert torch.equal(a, b.cpu()), name
 
 
+@pytest.mark.parametrize("Z,H,L", [(12, 24, 768), (100, 4, 1024)])
+def test_persistent_forward_many_items_per_block(Z, H, L):
+    """Head dimension 64 runs one persistent block per SM: with 12 samples the
+    blocks walk several length-ranked items each (one- and two-tile items
+    mixed), with 100 samples they walk the index-ordered grid and skip items
+    without work.  Every output row against the oracle."""
+    dev = _dev()
+    g = np.random.default_rng(Z + L)
+    nq = g.integers(0, L + 1, size=Z)
+    nk = g.integers(0, L + 1, size=Z)
+    nq[::9], nk[1::11] = 0, 0
+    nq[2], nk[2] = L, L
+    inp = _case(Z, L, H, 64, nq, nk, seed=8500 + Z)
+    _check_full(inp, _run(inp, dev), "bf16")
+
+
 @pytest.mark.parametrize("Z", [40, 70])
 def test_many_samples_launch_order(Z):
     """Up to 64 samples the kernels rank them by length with two samples per
