@@ -148,7 +148,8 @@ sigattn_status sigattn_bwd_rect(const void *q, const void *k, const void *v, con
  * overlapped.  The batch is cut into units of one sample and a group of heads
  * (about 16 units in all, so that the first copy in and the last copy out,
  * which nothing overlaps, are short, but never less than 8 MB per tensor of a
- * unit, so that whole samples stay whole when they are small).
+ * unit, so that whole samples stay whole when they are small; the first and
+ * the last group are then halved, as nothing overlaps their copies).
  * Per unit, its rows of q, k, v, dout (host, [Z][L][H][D]) are copied into a
  * compact device slot on a library-owned copy stream while earlier units
  * compute; the forward and the backward of the unit run on one of two

@@ -579,9 +579,43 @@ sigattn_status sigattn_fwd_bwd_host(const void *q, const void *k, const void *v,
     if (cudaEventRecord(hp->start, st) != cudaSuccess) return cuda_fail();
     for (cudaStream_t x : {hp->in, hp->out, hp->comp[0], hp->comp[1]})
         if (cudaStreamWaitEvent(x, hp->start, 0) != cudaSuccess) return cuda_fail();
-    const int units = Z * chunks;
+    // Units in order: sample-major, head groups of up to hpu heads.  Nothing
+    // overlaps the first unit's copy in or the last unit's copy out, so those
+    // two groups are halved (when they hold two heads or more).
+    struct Unit {
+        int z, h0, hc;
+    };
+    auto unit_at = [&](int i) -> Unit {
+        // i-th unit of the plain list (before halving)
+        const int z = i / chunks, h0 = (i % chunks) * hpu;
+        return Unit{z, h0, std::min(hpu, H - h0)};
+    };
+    const int plain = Z * chunks;
+    const bool split_first = plain >= 2 && unit_at(0).hc >= 2;
+    const bool split_last = plain >= 2 && unit_at(plain - 1).hc >= 2;
+    const int units = plain + (split_first ? 1 : 0) + (split_last ? 1 : 0);
+    auto unit = [&](int u) -> Unit {
+        if (split_first) {
+            if (u == 0) {
+                const Unit a = unit_at(0);
+                return Unit{a.z, a.h0, a.hc / 2};
+            }
+            if (u == 1) {
+                const Unit a = unit_at(0);
+                return Unit{a.z, a.h0 + a.hc / 2, a.hc - a.hc / 2};
+            }
+            --u;
+        }
+        if (split_last && u >= plain - 1) {
+            const Unit b = unit_at(plain - 1);
+            return u == plain - 1 ? Unit{b.z, b.h0, b.hc / 2}
+                                  : Unit{b.z, b.h0 + b.hc / 2, b.hc - b.hc / 2};
+        }
+        return unit_at(u);
+    };
     for (int u = 0; u < units; ++u) {
-        const int z = u / chunks, h0 = (u % chunks) * hpu, hc = std::min(hpu, H - h0);
+        const Unit un = unit(u);
+        const int z = un.z, h0 = un.h0, hc = un.hc;
         const int slot = u % kPipeSlots;
         cudaStream_t cs = hp->comp[u & 1];
         uint8_t *base = ws + static_cast<size_t>(slot) * 8 * slot_tensor;

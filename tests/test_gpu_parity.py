@@ -315,6 +315,44 @@ def test_host_buffer_pipeline_matches_device_path(Z, L, H, D, dtype):
         assert torch.equal(a, b.cpu()), name
 
 
+def _random_case(seed):
+    """A seeded random problem: 1-90 samples (ranked by length or in index
+    order), 1-6 heads, a padded length that is rarely a multiple of 128, and
+    lengths that include 0, 1 and L; small enough for the oracle to check every
+    row in about a second."""
+    g = np.random.default_rng(seed)
+    D = int(g.choice([64, 128]))
+    Z = int(g.choice([1, 2, 3, 5, 8, 17, 40, 64, 65, 90]))
+    H = int(g.integers(1, 7))
+    budget = 2.5e7 / (Z * H)                    # valid (query, key) pairs at most
+    L = int(min(1200, max(60, np.sqrt(budget) * g.uniform(0.5, 1.5))))
+    nq = g.integers(0, L + 1, size=Z)
+    nk = g.integers(0, L + 1, size=Z)
+    for arr in (nq, nk):
+        arr[g.integers(0, Z)] = L
+        if Z > 2:
+            arr[g.integers(0, Z)] = 0
+            arr[g.integers(0, Z)] = 1
+    mode = "tanh" if g.integers(0, 2) == 0 else "exp"
+    return Z, L, H, D, nq, nk, mode
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_shapes_full(seed):
+    """Seeded random shapes and lengths (both head dimensions, both sigma forms,
+    more and fewer than 64 samples): every output row against the oracle."""
+    dev = _dev()
+    Z, L, H, D, nq, nk, mode = _random_case(9000 + seed)
+    inp = _case(Z, L, H, D, nq, nk, seed=9100 + seed)
+    old = sa.get_sigmoid_mode()
+    sa.set_sigmoid_mode(sa.SIGMOID_TANH if mode == "tanh" else sa.SIGMOID_EXP)
+    try:
+        outs = _run(inp, dev)
+    finally:
+        sa.set_sigmoid_mode(old)
+    _check_full(inp, outs, "bf16")
+
+
 @pytest.mark.parametrize("Z,H,L", [(12, 24, 768), (100, 4, 1024)])
 def test_persistent_forward_many_items_per_block(Z, H, L):
     """Head dimension 64 runs one persistent block per SM: with 12 samples the
