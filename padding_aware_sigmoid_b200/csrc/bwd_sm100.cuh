@@ -7,15 +7,15 @@
 //
 // Both kernels share the forward's structure: warps 0 and 2 issue TMA loads
 // (one ring each), warp 1 issues tcgen05.mma (running converged, one elected
-// lane issuing), and two warpgroups (warps 4-7 and 8-11) turn the fp32 score
-// tiles in TMEM into bf16 operands, each owning 64 of the 128 columns (thread =
-// TMEM lane = tile row).  The bf16 results are
-// written back into TMEM over columns their own warpgroup has already read,
-// and become the TMEM-resident A operand of the next MMA:
-//   warpgroup 0 writes packed columns [base, base+32)     for tile columns 0..63
-//   warpgroup 1 writes packed columns [base+64, base+96)  for tile columns 64..127
-// so the MMA step kk (16 tile columns) reads TMEM column
-//   base + (kk < 4 ? 8 kk : 64 + 8 (kk - 4)).
+// lane issuing), and four warpgroups (warps 4-19) turn the fp32 score tiles in
+// TMEM into bf16 operands, warpgroup w owning tile columns [32 w, 32 w + 32)
+// (thread = TMEM lane = tile row).  Four warps per SM sub-partition keep the
+// MUFU at its full rate and split each step's element-wise work four ways.
+// The bf16 results are written back into TMEM over columns their own
+// warpgroup has already read, and become the TMEM-resident A operand of the
+// next MMA: warpgroup w writes packed columns [base + 32 w, base + 32 w + 16)
+// for its 32 tile columns, so the MMA step kk (16 tile columns) reads TMEM
+// column base + 32 (kk / 2) + 8 (kk % 2).
 // The warpgroups hand their work over in two steps (first what depends on
 // the scores only, then what needs dP), so that the next scores' MMA runs
 // while the warpgroups still work on the current tile.
@@ -61,8 +61,8 @@ struct BwdLayout {
     static constexpr int NBAR = 1 + 2 * SX + 2 * SY + MAX_HANDOFF;
     static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM + 8;
-    static constexpr int OFF_RED = OFF_ABORT + 8;      // 8 floats: per-warp db partials
-    static constexpr int OFF_SAMPLE = OFF_RED + 32;    // this block's sample and lengths
+    static constexpr int OFF_RED = OFF_ABORT + 8;      // 16 floats: per-warp db partials
+    static constexpr int OFF_SAMPLE = OFF_RED + 64;    // this block's sample and lengths
     static constexpr int SMEM_ALLOC = OFF_SAMPLE + 16 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
@@ -95,7 +95,39 @@ __device__ __forceinline__ void ring_drain(uint64_t *full, int issued, uint64_t 
         mbar_wait_drain(&full[j % S], (j / S) & 1, limit_ns);
 }
 
-__device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
+// Sigma warpgroups per backward block.  At D = 64 a tile's sigma' work is
+// twice its MMA work and four warpgroups (32 tile columns each) keep up with
+// the tensor core; at D = 128 the two are equal and two warpgroups (64 columns
+// each, with more registers per thread) measured faster.
+template <int D>
+struct BwdSigma {
+    static constexpr int NG = D == 64 ? 4 : 2;
+    static constexpr int kThreads = 128 + 128 * NG;
+    static constexpr int kCols = 128 / NG;       // tile columns per warpgroup
+    static constexpr int kPacked = kCols / 2;    // TMEM columns of their bf16 pairs
+    static constexpr int kArrivals = 128 * NG;   // one per sigma thread
+    // TMEM column (relative to the buffer) of the packed bf16 values of K step
+    // kk (tile columns 16 kk .. 16 kk + 15), which warpgroup 16 kk / kCols wrote
+    // over the first kPacked of its own columns.
+    static __device__ __forceinline__ uint32_t packed_col(int kk) {
+        return kCols * ((16 * kk) / kCols) + ((16 * kk) % kCols) / 2;
+    }
+};
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 16 || N == 32 || N == 64, "column count");
+    if constexpr (N == 16) tmem_ld16(taddr, r);
+    else if constexpr (N == 32) tmem_ld32(taddr, r);
+    else tmem_ld64(taddr, r);
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+    static_assert(N == 16 || N == 32, "column count");
+    if constexpr (N == 16) tmem_st16(taddr, r);
+    else tmem_st32(taddr, r);
+}
 
 // Stores one row of D fp32 accumulator columns from TMEM as bf16, scaled by
 // `scale`, or zeros when !valid.  All 32 lanes of the warp must call it.
@@ -134,11 +166,12 @@ __device__ __forceinline__ void zero_rows(__nv_bfloat16 *base, int z, int h, int
     }
 }
 
-// Packs 32 pairs to bf16 and zeroes the entries at tile columns >= valid
-// (columns [col0, col0 + 64) of the tile; valid = count of in-range columns).
-__device__ __forceinline__ void mask_packed(uint32_t (&pk)[32], int col0, int valid) {
+// Zeroes the packed bf16 pairs at tile columns >= valid (pk holds columns
+// [col0, col0 + 2 N) of the tile; valid = count of in-range columns).
+template <int N>
+__device__ __forceinline__ void mask_packed(uint32_t (&pk)[N], int col0, int valid) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < N; ++i) {
         const int c = col0 + 2 * i;
         const uint32_t lo = c < valid ? 0x0000FFFFu : 0u;
         const uint32_t hi = c + 1 < valid ? 0xFFFF0000u : 0u;
@@ -156,17 +189,19 @@ __device__ __forceinline__ void mask_packed(uint32_t (&pk)[32], int col0, int va
 // over dP_j.  The MMA thread issues S_{j+1} as soon as S_j is released and
 // dP_{j+1} into the other dP buffer (its dS_{j-1} is read by an earlier MMA of
 // the same thread, and MMAs run in issue order), then dQ += dS_j K_j when dS_j
-// is ready: neither warpgroup phase waits on the MMA of the previous tile.  Both
-// warpgroups run their sigma' phase at the same time, so that two warps share
-// each SM sub-partition's MUFU (one warp alone leaves it idle between issues).
+// is ready: neither warpgroup phase waits on the MMA of the previous tile.  The
+// NG warpgroups (each with kCols tile columns) run their sigma' phase at the
+// same time, so that NG warps share each SM sub-partition's MUFU (one warp
+// alone leaves it idle between issues).
 // ============================================================================
 // DB: also accumulate the bias gradient (p.db_part must then be set)
 template <int D, int MODE, int SX, int SY, bool DB>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BwdParams p) {
     using Lay = BwdLayout<D, SX, SY>;
+    using SG = BwdSigma<D>;
     constexpr uint32_t kColS = 0, kColDP0 = 128, kColDP1 = 256, kColDQ = 384;
     static_assert(kColDQ + D <= Lay::TMEM_COLS, "TMEM budget");
     extern __shared__ uint8_t smem_raw[];
@@ -226,9 +261,9 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(s_full, 1);
         mbar_init(&dp_full[0], 1);
         mbar_init(&dp_full[1], 1);
-        mbar_init(s_free, 256);
-        mbar_init(&ds_ready[0], 256);
-        mbar_init(&ds_ready[1], 256);
+        mbar_init(s_free, BwdSigma<D>::kArrivals);
+        mbar_init(&ds_ready[0], BwdSigma<D>::kArrivals);
+        mbar_init(&ds_ready[1], BwdSigma<D>::kArrivals);
         mbar_init(dq_done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -336,7 +371,7 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t sK = kslot(j);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts_w(tmem + kColDQ, tmem + dcol + packed_col(kk),
+                    mma_ts_w(tmem + kColDQ, tmem + dcol + BwdSigma<D>::packed_col(kk),
                              smem_desc_sw128(sK + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_q,
                              (j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit_w(&x_empty[j % SX]);           // K_j: S_j and dQ_j done
@@ -346,7 +381,7 @@ __global__ void __launch_bounds__(384, 1)
             __syncwarp();
         }
     } else if (warp >= 4) {
-        const int w = (warp - 4) >> 2;      // warpgroup: tile columns [64w, 64w+64)
+        const int w = (warp - 4) >> 2;      // warpgroup: tile columns [kCols w, kCols (w + 1))
         const int quarter = warp & 3;
         const int row = qtile * 128 + quarter * 32 + lane;
         const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
@@ -357,75 +392,79 @@ __global__ void __launch_bounds__(384, 1)
         {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             for (int j = 0; j < nkv; ++j) {
-                float2 g[32];
+                float2 g[SG::kPacked];
                 {
-                    if (quarter == 0) trace(2 + w, j, 0);
+                    if (quarter == 0) trace(2 + (w & 1), j, 0);
                     ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, wctx));
                     if (!ok) break;
-                    if (quarter == 0) trace(2 + w, j, 1);
+                    if (quarter == 0) trace(2 + (w & 1), j, 1);
                     tc_fence_after();
-                    uint32_t r[64];
-                    tmem_ld64(tmem + lane_bits + kColS + 64 * w, r);
-                    if (quarter == 0) trace(2 + w, j, 2);
+                    uint32_t r[SG::kCols];
+                    tmem_ld_cols(tmem + lane_bits + kColS + SG::kCols * w, r);
+                    if (quarter == 0) trace(2 + (w & 1), j, 2);
                     tc_fence_before();
                     mbar_arrive(s_free);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < SG::kPacked; ++i) {
                         float2 pr;
                         sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf),
                                           pr, g[i]);
                     }
                 }
-                const uint32_t dcol = (j & 1 ? kColDP1 : kColDP0) + 64 * w;
-                if (quarter == 0) trace(2 + w, j, 3);
+                const uint32_t dcol = (j & 1 ? kColDP1 : kColDP0) + SG::kCols * w;
+                if (quarter == 0) trace(2 + (w & 1), j, 3);
                 ok = __all_sync(0xffffffffu, mbar_wait(&dp_full[j & 1], (j >> 1) & 1, wctx));
                 if (!ok) break;
-                if (quarter == 0) trace(2 + w, j, 4);
+                if (quarter == 0) trace(2 + (w & 1), j, 4);
                 tc_fence_after();
-                uint32_t d[64];
-                tmem_ld64(tmem + lane_bits + dcol, d);
-                if (quarter == 0) trace(2 + w, j, 5);
-                uint32_t pk[32];
+                uint32_t d[SG::kCols];
+                tmem_ld_cols(tmem + lane_bits + dcol, d);
+                if (quarter == 0) trace(2 + (w & 1), j, 5);
+                uint32_t pk[SG::kPacked];
                 const int kvalid = nk - j * 128;
                 float2 dsum = f2(0.0f, 0.0f);   // this row's fp32 dS over keys below n_k
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < SG::kPacked; ++i) {
                     const float2 ds = mul2(g[i], f2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
                     pk[i] = pack_bf16x2(ds.x, ds.y);
                     if constexpr (DB) {
-                        const int c = 64 * w + 2 * i;
+                        const int c = SG::kCols * w + 2 * i;
                         dsum.x += c < kvalid ? ds.x : 0.0f;
                         dsum.y += c + 1 < kvalid ? ds.y : 0.0f;
                     }
                 }
                 if constexpr (DB) dbacc += dsum.x + dsum.y;
-                if (kvalid < 128) mask_packed(pk, 64 * w, kvalid);
-                tmem_st32(tmem + lane_bits + dcol, pk);
+                if (kvalid < 128) mask_packed(pk, SG::kCols * w, kvalid);
+                // dS over the first kPacked of this warpgroup's dP columns, just read
+                tmem_st_cols(tmem + lane_bits + dcol, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&ds_ready[j & 1]);
-                if (quarter == 0) trace(2 + w, j, 6);
+                if (quarter == 0) trace(2 + (w & 1), j, 6);
             }
             // every MMA of this CTA has finished once the MMA thread's final commit lands
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
-            if (ok) {
+            // dQ's D columns split over the warpgroups, at least 32 each (with
+            // four warpgroups at D = 64 the last two have none)
+            constexpr int kEpi = D / SG::NG >= 32 ? D / SG::NG : 32;
+            if (ok && w * kEpi < D) {
                 tc_fence_after();
                 store_row_from_tmem<D>(tmem + lane_bits + kColDQ, drow, row < L, row < nq,
-                                       p.alpha, w * (D / 2), D / 2);
+                                       p.alpha, w * kEpi, kEpi);
             }
         }
         if constexpr (DB) {
             // one partial per CTA, summed in a fixed order: warp sums, then the
-            // eight warps' sums in warp order (rows at or beyond n_q add nothing)
+            // 4 NG warps' sums in warp order (rows at or beyond n_q add nothing)
             float v = row < nq ? dbacc : 0.0f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             float *red = reinterpret_cast<float *>(smem + Lay::OFF_RED);
             if (lane == 0) red[warp - 4] = v;
-            sigma_warps_sync(256);
+            sigma_warps_sync(SG::kArrivals);
             if (warp == 4 && lane == 0) {
                 float t = 0.0f;
-                for (int u = 0; u < 8; ++u) t += red[u];
+                for (int u = 0; u < 4 * SG::NG; ++u) t += red[u];
                 p.db_part[(static_cast<size_t>(z) * p.H + h) * gridDim.x + qtile] = t;
             }
         }
@@ -444,26 +483,27 @@ __global__ void __launch_bounds__(384, 1)
 // ============================================================================
 // dK/dV kernel: one CTA per 128-key tile; streams Q_i, dO_i for i < ceil(n_q/128).
 // Works on the transposed scores (rows = keys):
-//   S^T = K Q_i^T, dP^T = V dO_i^T, P^T -> TMEM over S^T, dS^T -> TMEM over dP^T,
+//   S^T = K Q_i^T, dP^T = V dO_i^T, P^T and dS^T -> TMEM over dP^T,
 //   dV += P^T dO_i, dK += dS^T Q_i.
 // TMEM: [0,128) S^T, [128,256) dP^T, then P^T and dS^T over it,
 // [256,256+D) dV, [256+D,256+2D) dK.
 //
-// A warpgroup reads its 64 columns of S^T into registers and releases the S^T
-// buffer at once, so S^T_{i+1} is computed while it evaluates sigma and
-// sigma' for tile i.  It keeps P^T in registers until it has read its dP^T
-// columns, then writes P^T over the first 32 of them (tile columns 64w..64w+63
-// packed two per column) and dS^T over the other 32.  MMA order per query
+// A warpgroup reads its kCols columns of S^T into registers and releases the
+// S^T buffer at once, so S^T_{i+1} is computed while it evaluates sigma and
+// sigma' for tile i.  It keeps P^T in registers until it has read the first
+// half of its dP^T columns, then writes P^T over them (its kCols tile columns
+// packed two per TMEM column) and dS^T over the other half.  MMA order per query
 // tile: S^T_{i+1} (as soon as S^T_i is read), dV_i, dK_i, dP^T_{i+1} (over P^T_i
 // and dS^T_i, read by dV_i and dK_i just before: MMAs from one thread run in
 // issue order).
 // ============================================================================
 template <int D, int MODE, int SX, int SY>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const BwdParams p) {
     using Lay = BwdLayout<D, SX, SY>;
+    using SG = BwdSigma<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::OFF_BAR);
@@ -518,9 +558,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(s_free, 256);
-        mbar_init(p_ready, 256);
-        mbar_init(ds_ready, 256);
+        mbar_init(s_free, BwdSigma<D>::kArrivals);
+        mbar_init(p_ready, BwdSigma<D>::kArrivals);
+        mbar_init(ds_ready, BwdSigma<D>::kArrivals);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -597,7 +637,7 @@ __global__ void __launch_bounds__(384, 1)
             auto issue_acc = [&](uint32_t acc, uint32_t acol, uint32_t bbase, bool first) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts_w(tmem + acc, tmem + acol + packed_col(kk),
+                    mma_ts_w(tmem + acc, tmem + acol + BwdSigma<D>::packed_col(kk),
                              smem_desc_sw128(bbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_kv,
                              (!first || kk > 0) ? 1u : 0u);
             };
@@ -628,7 +668,7 @@ __global__ void __launch_bounds__(384, 1)
                 if (!(ok = wait(ds_ready, i & 1))) break;
                 if (lane == 0) trace(1, i, 2);
                 tc_fence_after();
-                issue_acc(Lay::COL_ACC1, Lay::COL_DP + 32, qslot(i), i == 0);  // dK += dS^T Q_i
+                issue_acc(Lay::COL_ACC1, Lay::COL_DP + SG::kPacked, qslot(i), i == 0);  // dK += dS^T Q_i
                 mma_commit_w(&x_empty[i % SX]);                                 // Q_i: S^T_i, dK_i done
                 if (more) {
                     // dP^T_{i+1} overwrites P^T_i and dS^T_i, read by the two MMAs just
@@ -645,55 +685,59 @@ __global__ void __launch_bounds__(384, 1)
             __syncwarp();
         }
     } else if (warp >= 4) {
-        const int w = (warp - 4) >> 2;      // warpgroup: query columns [64w, 64w+64)
+        const int w = (warp - 4) >> 2;      // warpgroup: query columns [kCols w, kCols (w + 1))
         const int quarter = warp & 3;
         const int row = ktile * 128 + quarter * 32 + lane;   // key row
         const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
         const size_t roff = (static_cast<size_t>(z) * L + row) * (static_cast<size_t>(p.H) * D) +
                             static_cast<size_t>(h) * D;
-        __nv_bfloat16 *dst = (w == 0 ? p.dv : p.dk) + roff;
+        // epilogue: the first half of the warpgroups writes dV, the second dK,
+        // D / kOut columns each
+        constexpr int kOut = SG::NG / 2;
+        const bool is_dv = w < kOut;
+        __nv_bfloat16 *dst = (is_dv ? p.dv : p.dk) + roff;
         bool ok = true;
         {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
-            const uint32_t tS = tmem + lane_bits + Lay::COL_S + 64 * w;
-            const uint32_t tD = tmem + lane_bits + Lay::COL_DP + 64 * w;
+            const uint32_t tS = tmem + lane_bits + Lay::COL_S + SG::kCols * w;
+            const uint32_t tD = tmem + lane_bits + Lay::COL_DP + SG::kCols * w;
             for (int i = 0; i < nqt; ++i) {
                 const int qvalid = nq - i * 128;
-                float2 g[32];
-                uint32_t pk[32];
-                if (quarter == 0) trace(2 + w, i, 0);
+                float2 g[SG::kPacked];
+                uint32_t pk[SG::kPacked];
+                if (quarter == 0) trace(2 + (w & 1), i, 0);
                 ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
                 if (!ok) break;
-                if (quarter == 0) trace(2 + w, i, 1);
+                if (quarter == 0) trace(2 + (w & 1), i, 1);
                 tc_fence_after();
                 {
-                    uint32_t r[64];
-                    tmem_ld64(tS, r);
+                    uint32_t r[SG::kCols];
+                    tmem_ld_cols(tS, r);
                     // S^T_i is in registers: the MMA warp may compute S^T_{i+1} now
                     tc_fence_before();
                     mbar_arrive(s_free);
 #pragma unroll
-                    for (int ii = 0; ii < 32; ++ii) {
+                    for (int ii = 0; ii < SG::kPacked; ++ii) {
                         float2 pr;
                         sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * ii]), __uint_as_float(r[2 * ii + 1]), cf),
                                           pr, g[ii]);
                         pk[ii] = pack_bf16x2(pr.x, pr.y);
                     }
                 }
-                if (qvalid < 128) mask_packed(pk, 64 * w, qvalid);
-                if (quarter == 0) trace(2 + w, i, 2);
+                if (qvalid < 128) mask_packed(pk, SG::kCols * w, qvalid);
+                if (quarter == 0) trace(2 + (w & 1), i, 2);
                 ok = __all_sync(0xffffffffu, mbar_wait(dp_full, i & 1, wctx));
                 if (!ok) break;
-                if (quarter == 0) trace(2 + w, i, 3);
+                if (quarter == 0) trace(2 + (w & 1), i, 3);
                 tc_fence_after();
-                uint32_t ds[32];
+                uint32_t ds[SG::kPacked];
                 {
-                    // first 32 dP^T columns, then P^T over them
-                    uint32_t d[32];
-                    tmem_ld32(tD, d);
-                    tmem_st32(tD, pk);
+                    // the first kPacked of this warpgroup's dP^T columns, then P^T over them
+                    uint32_t d[SG::kPacked];
+                    tmem_ld_cols(tD, d);
+                    tmem_st_cols(tD, pk);
 #pragma unroll
-                    for (int ii = 0; ii < 16; ++ii) {
+                    for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
                         const float2 v = mul2(g[ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
                         ds[ii] = pack_bf16x2(v.x, v.y);
                     }
@@ -702,28 +746,30 @@ __global__ void __launch_bounds__(384, 1)
                     mbar_arrive(p_ready);
                 }
                 {
-                    // the other 32 dP^T columns, then dS^T over them
-                    uint32_t d[32];
-                    tmem_ld32(tD + 32, d);
+                    // the other kPacked dP^T columns, then dS^T over them
+                    uint32_t d[SG::kPacked];
+                    tmem_ld_cols(tD + SG::kPacked, d);
 #pragma unroll
-                    for (int ii = 0; ii < 16; ++ii) {
-                        const float2 v = mul2(g[16 + ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
-                        ds[16 + ii] = pack_bf16x2(v.x, v.y);
+                    for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
+                        const float2 v = mul2(g[SG::kPacked / 2 + ii],
+                                              f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
+                        ds[SG::kPacked / 2 + ii] = pack_bf16x2(v.x, v.y);
                     }
                 }
-                if (qvalid < 128) mask_packed(ds, 64 * w, qvalid);
-                tmem_st32(tD + 32, ds);
+                if (qvalid < 128) mask_packed(ds, SG::kCols * w, qvalid);
+                tmem_st_cols(tD + SG::kPacked, ds);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ds_ready);
-                if (quarter == 0) trace(2 + w, i, 4);
+                if (quarter == 0) trace(2 + (w & 1), i, 4);
             }
             // every MMA of this CTA has finished once the MMA thread's final commit lands
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
             if (ok) {
                 tc_fence_after();
-                store_row_from_tmem<D>(tmem + lane_bits + (w == 0 ? Lay::COL_ACC0 : Lay::COL_ACC1), dst,
-                                       row < L, row < nk, w == 0 ? 1.0f : p.alpha, 0, D);
+                store_row_from_tmem<D>(tmem + lane_bits + (is_dv ? Lay::COL_ACC0 : Lay::COL_ACC1), dst,
+                                       row < L, row < nk, is_dv ? 1.0f : p.alpha, (w % kOut) * (D / kOut),
+                                       D / kOut);
             }
         }
     }

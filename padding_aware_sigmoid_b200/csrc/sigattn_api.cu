@@ -317,14 +317,14 @@ sigattn_status bwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
     if (parts & kPartDq) {
         sigattn_status s =
             p.db_part != nullptr
-                ? launch(bwd_dq_kernel<D, MODE, SX, SY, true>, grid, dim3(384), smem, st, mq, mk,
+                ? launch(bwd_dq_kernel<D, MODE, SX, SY, true>, grid, dim3(BwdSigma<D>::kThreads), smem, st, mq, mk,
                          mv, mdo, p)
-                : launch(bwd_dq_kernel<D, MODE, SX, SY, false>, grid, dim3(384), smem, st, mq, mk,
+                : launch(bwd_dq_kernel<D, MODE, SX, SY, false>, grid, dim3(BwdSigma<D>::kThreads), smem, st, mq, mk,
                          mv, mdo, p);
         if (s != SIGATTN_OK) return s;
     }
     if (parts & kPartDkdv)
-        return launch(bwd_dkdv_kernel<D, MODE, SX, SY>, grid_kv, dim3(384), smem, st, mq, mk, mv,
+        return launch(bwd_dkdv_kernel<D, MODE, SX, SY>, grid_kv, dim3(BwdSigma<D>::kThreads), smem, st, mq, mk, mv,
                       mdo, p);
     return SIGATTN_OK;
 }
