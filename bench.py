@@ -637,15 +637,24 @@ TRAFFIC_KERNELS = {"fwd": "fwd_tiles_kernel", "bwd_dq": "bwd_dq_kernel",
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")
 
 
-def kernel_source_hash() -> str:
-    """sha256 over the device-code headers of the library (names and contents)."""
+def _code_tokens(text: str) -> str:
+    """C++ source with comments removed and whitespace runs collapsed: what the
+    compiler sees (string literals in these headers hold no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def kernel_source_hash(src: str = "") -> str:
+    """sha256 over the device-code headers of the library (names and code, with
+    comments and layout ignored, so an edit of comments keeps the captures)."""
     import hashlib
     h = hashlib.sha256()
-    src = os.path.join(ROOT, "padding_aware_sigmoid_b200", "csrc")
+    src = src or os.path.join(ROOT, "padding_aware_sigmoid_b200", "csrc")
     for name in DEVICE_SOURCES:
         h.update(name.encode())
-        with open(os.path.join(src, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(src, name), encoding="utf-8") as f:
+            h.update(_code_tokens(f.read()).encode())
     return h.hexdigest()
 
 

@@ -7,15 +7,15 @@
 //
 // Both kernels share the forward's structure: warps 0 and 2 issue TMA loads
 // (one ring each), warp 1 issues tcgen05.mma (running converged, one elected
-// lane issuing), and four warpgroups (warps 4-19) turn the fp32 score tiles in
-// TMEM into bf16 operands, warpgroup w owning tile columns [32 w, 32 w + 32)
-// (thread = TMEM lane = tile row).  Four warps per SM sub-partition keep the
-// MUFU at its full rate and split each step's element-wise work four ways.
-// The bf16 results are written back into TMEM over columns their own
-// warpgroup has already read, and become the TMEM-resident A operand of the
-// next MMA: warpgroup w writes packed columns [base + 32 w, base + 32 w + 16)
-// for its 32 tile columns, so the MMA step kk (16 tile columns) reads TMEM
-// column base + 32 (kk / 2) + 8 (kk % 2).
+// lane issuing), and NG sigma warpgroups (warps 4 and up; NG = 2 at D = 128,
+// 4 at D = 64, see BwdSigma) turn the fp32 score tiles in TMEM into bf16
+// operands, warpgroup w owning the kCols = 128 / NG tile columns
+// [kCols w, kCols (w + 1)) (thread = TMEM lane = tile row).  The bf16 results
+// are written back into TMEM over columns their own warpgroup has already
+// read, and become the TMEM-resident A operand of the next MMA: warpgroup w
+// writes its kCols tile columns packed two per TMEM column at
+// [base + kCols w, base + kCols w + kCols / 2), so the MMA step kk (16 tile
+// columns) reads the TMEM column BwdSigma<D>::packed_col(kk) past base.
 // The warpgroups hand their work over in two steps (first what depends on
 // the scores only, then what needs dP), so that the next scores' MMA runs
 // while the warpgroups still work on the current tile.

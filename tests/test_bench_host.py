@@ -77,6 +77,24 @@ def test_traffic_written_from_ncu_csv_carries_the_device_code_hash(tmp_path, mon
     assert bench._ncu_traffic("fwd") is None
 
 
+def test_device_code_hash_ignores_comments_but_not_code(tmp_path):
+    """The traffic captures stay valid across comment edits of the device
+    headers and are voided by any change of the code itself."""
+    src = os.path.join(bench.ROOT, "padding_aware_sigmoid_b200", "csrc")
+    base = bench.kernel_source_hash(src)
+    for variant, same in (("comment", True), ("code", False)):
+        d = tmp_path / variant
+        d.mkdir()
+        for name in bench.DEVICE_SOURCES:
+            with open(os.path.join(src, name), encoding="utf-8") as f:
+                text = f.read()
+            if name == "sigmoid.cuh":
+                text = ("// an added comment line\n/* and a block\n comment */" + text
+                        if variant == "comment" else text.replace("0.5f", "0.25f", 1))
+            (d / name).write_text(text, encoding="utf-8")
+        assert (bench.kernel_source_hash(str(d)) == base) == same, variant
+
+
 def test_gpus_2_starts_two_ranks_and_reports_them():
     """`bench.py --gpus 2` outside torchrun starts two ranks itself; on the
     reference arm rank 0 alone times the oracle and prints the line, and the
