@@ -16,9 +16,8 @@
 // writes its kCols tile columns packed two per TMEM column at
 // [base + kCols w, base + kCols w + kCols / 2), so the MMA step kk (16 tile
 // columns) reads the TMEM column BwdSigma<D>::packed_col(kk) past base.
-// The warpgroups hand their work over in two steps (first what depends on
-// the scores only, then what needs dP), so that the next scores' MMA runs
-// while the warpgroups still work on the current tile.
+// The warpgroups release each score buffer as soon as they have read it, so
+// that the next scores' MMA runs while they still work on the current tile.
 #pragma once
 
 #include "sm100.cuh"
@@ -184,15 +183,18 @@ __device__ __forceinline__ void mask_packed(uint32_t (&pk)[N], int col0, int val
 // TMEM: [0,128) S, [128,256) and [256,384) dP of even / odd key tiles (each
 // overwritten by its dS, bf16 packed), [384,384+D) dQ.
 //
-// Per key tile j the warpgroups (1) read S_j and release it, keeping
-// sigma'(S_j) in registers, then (2) read dP_j and write dS_j = sigma' dP_j
-// over dP_j.  The MMA thread issues S_{j+1} as soon as S_j is released and
-// dP_{j+1} into the other dP buffer (its dS_{j-1} is read by an earlier MMA of
-// the same thread, and MMAs run in issue order), then dQ += dS_j K_j when dS_j
-// is ready: neither warpgroup phase waits on the MMA of the previous tile.  The
-// NG warpgroups (each with kCols tile columns) run their sigma' phase at the
-// same time, so that NG warps share each SM sub-partition's MUFU (one warp
-// alone leaves it idle between issues).
+// Per key tile j the warpgroups read S_j into registers and release it, then
+// read dP_j 32 columns at a time and write dS_j = sigma'(S_j) dP_j over it,
+// forming sigma' and dS in one pass so that the MUFU work of one chunk
+// overlaps the multiplies and bf16 packing of the other (done one after the
+// other, the two phases took ~1000 and ~490 clk per tile at D = 128).  The
+// MMA thread issues S_{j+1} as soon as S_j is released and dP_{j+1} right
+// after it into the other dP buffer (its dS_{j-1} is read by an earlier MMA of
+// the same thread, and MMAs run in issue order), so both are ready when the
+// warpgroups reach tile j+1; dQ += dS_j K_j follows when dS_j is ready.  The
+// NG warpgroups (each with kCols tile columns) work on a tile at the same
+// time, so that NG warps share each SM sub-partition's MUFU (one warp alone
+// leaves it idle between issues).
 // ============================================================================
 // DB: also accumulate the bias gradient (p.db_part must then be set)
 template <int D, int MODE, int SX, int SY, bool DB>
@@ -392,24 +394,29 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
         {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             for (int j = 0; j < nkv; ++j) {
-                float2 g[SG::kPacked];
-                {
-                    if (quarter == 0) trace(2 + (w & 1), j, 0);
-                    ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, wctx));
-                    if (!ok) break;
-                    if (quarter == 0) trace(2 + (w & 1), j, 1);
-                    tc_fence_after();
-                    uint32_t r[SG::kCols];
-                    tmem_ld_cols(tmem + lane_bits + kColS + SG::kCols * w, r);
-                    if (quarter == 0) trace(2 + (w & 1), j, 2);
-                    tc_fence_before();
-                    mbar_arrive(s_free);
+                if (quarter == 0) trace(2 + (w & 1), j, 0);
+                ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, wctx));
+                if (!ok) break;
+                if (quarter == 0) trace(2 + (w & 1), j, 1);
+                tc_fence_after();
+                uint32_t r[SG::kCols];
+                tmem_ld_cols(tmem + lane_bits + kColS + SG::kCols * w, r);
+                if (quarter == 0) trace(2 + (w & 1), j, 2);
+                tc_fence_before();
+                mbar_arrive(s_free);
+                // sigma'(S_j) and dS_j = sigma' dP_j are formed 32 columns at a
+                // time, so that the MUFU work of one chunk overlaps the multiplies
+                // and bf16 packing of the other.  With two chunks (64 columns per
+                // warpgroup) the first chunk's sigma' is taken before dP_j is
+                // waited for, covering the time dP_j may still need.
+                constexpr int kChunks = SG::kCols / 32;
+                constexpr int kPre = kChunks > 1 ? 1 : 0;   // chunks of sigma' before the dP wait
+                float2 gpre[16 * kPre + 1];
 #pragma unroll
-                    for (int i = 0; i < SG::kPacked; ++i) {
-                        float2 pr;
-                        sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf),
-                                          pr, g[i]);
-                    }
+                for (int i = 0; i < 16 * kPre; ++i) {
+                    float2 pr;
+                    sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf), pr,
+                                      gpre[i]);
                 }
                 const uint32_t dcol = (j & 1 ? kColDP1 : kColDP0) + SG::kCols * w;
                 if (quarter == 0) trace(2 + (w & 1), j, 3);
@@ -417,26 +424,39 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
                 if (!ok) break;
                 if (quarter == 0) trace(2 + (w & 1), j, 4);
                 tc_fence_after();
-                uint32_t d[SG::kCols];
-                tmem_ld_cols(tmem + lane_bits + dcol, d);
-                if (quarter == 0) trace(2 + (w & 1), j, 5);
-                uint32_t pk[SG::kPacked];
                 const int kvalid = nk - j * 128;
                 float2 dsum = f2(0.0f, 0.0f);   // this row's fp32 dS over keys below n_k
 #pragma unroll
-                for (int i = 0; i < SG::kPacked; ++i) {
-                    const float2 ds = mul2(g[i], f2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
-                    pk[i] = pack_bf16x2(ds.x, ds.y);
-                    if constexpr (DB) {
-                        const int c = SG::kCols * w + 2 * i;
-                        dsum.x += c < kvalid ? ds.x : 0.0f;
-                        dsum.y += c + 1 < kvalid ? ds.y : 0.0f;
+                for (int ch = 0; ch < kChunks; ++ch) {
+                    uint32_t d[32];
+                    tmem_ld32(tmem + lane_bits + dcol + 32 * ch, d);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float2 g;
+                        if (ch < kPre) {
+                            g = gpre[16 * ch + i];
+                        } else {
+                            float2 pr;
+                            sigma_grad2<MODE>(scale2(__uint_as_float(r[32 * ch + 2 * i]),
+                                                     __uint_as_float(r[32 * ch + 2 * i + 1]), cf),
+                                              pr, g);
+                        }
+                        const float2 ds = mul2(g, f2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
+                        pk[i] = pack_bf16x2(ds.x, ds.y);
+                        if constexpr (DB) {
+                            const int c = SG::kCols * w + 32 * ch + 2 * i;
+                            dsum.x += c < kvalid ? ds.x : 0.0f;
+                            dsum.y += c + 1 < kvalid ? ds.y : 0.0f;
+                        }
                     }
+                    if (kvalid < 128) mask_packed(pk, SG::kCols * w + 32 * ch, kvalid);
+                    // dS over the first kPacked of this warpgroup's dP columns: chunk
+                    // ch's 16 packed columns sit over dP columns this warpgroup has read
+                    tmem_st16(tmem + lane_bits + dcol + 16 * ch, pk);
                 }
+                if (quarter == 0) trace(2 + (w & 1), j, 5);
                 if constexpr (DB) dbacc += dsum.x + dsum.y;
-                if (kvalid < 128) mask_packed(pk, SG::kCols * w, kvalid);
-                // dS over the first kPacked of this warpgroup's dP columns, just read
-                tmem_st_cols(tmem + lane_bits + dcol, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&ds_ready[j & 1]);
