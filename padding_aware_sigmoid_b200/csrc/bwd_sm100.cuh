@@ -510,16 +510,22 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
 //   S^T = K Q_i^T, dP^T = V dO_i^T, P^T and dS^T -> TMEM over dP^T,
 //   dV += P^T dO_i, dK += dS^T Q_i.
 // TMEM: [0,128) S^T, [128,256) dP^T, then P^T and dS^T over it,
-// [256,256+D) dV, [256+D,256+2D) dK.
+// [256,256+D) dV, [256+D,256+2D) dK; at D = 64 a second dP^T buffer in
+// [384,512), the two alternating between query tiles.
 //
 // A warpgroup reads its kCols columns of S^T into registers and releases the
-// S^T buffer at once, so S^T_{i+1} is computed while it evaluates sigma and
-// sigma' for tile i.  It keeps P^T in registers until it has read the first
-// half of its dP^T columns, then writes P^T over them (its kCols tile columns
-// packed two per TMEM column) and dS^T over the other half.  MMA order per query
-// tile: S^T_{i+1} (as soon as S^T_i is read), dV_i, dK_i, dP^T_{i+1} (over P^T_i
-// and dS^T_i, read by dV_i and dK_i just before: MMAs from one thread run in
-// issue order).
+// S^T buffer at once, so S^T_{i+1} is computed while it works on tile i.  It
+// writes P^T (its kCols tile columns packed two per TMEM column) over the first
+// half of its dP^T columns once it has read them, and dS^T over the other half.
+// With one dP^T buffer (D = 128) it evaluates sigma and sigma' while dP^T_i is
+// still being computed, keeping P^T and sigma' in registers, and the MMA order
+// per query tile is S^T_{i+1} (as soon as S^T_i is read), dV_i, dK_i, dP^T_{i+1}
+// (over P^T_i and dS^T_i, read by dV_i and dK_i just before: MMAs from one
+// thread run in issue order).  With two (D = 64) dP^T_{i+1} follows S^T_{i+1}
+// at once, into the buffer of tile i-1 (whose readers dV_{i-1} and dK_{i-1}
+// were issued before), so dP^T_i is ready when the warpgroup starts tile i and
+// it forms P^T, sigma' and dS^T in one pass, 16 tile columns at a time, the
+// MUFU work of one chunk overlapping the packing of the other.
 // ============================================================================
 template <int D, int MODE, int SX, int SY>
 __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
