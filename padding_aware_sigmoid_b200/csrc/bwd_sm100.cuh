@@ -543,12 +543,19 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
     uint64_t *y_full = x_empty + SX;          // dO_i ring
     uint64_t *y_empty = y_full + SY;
     uint64_t *s_full = y_empty + SY;          // MMA -> WGs: S^T_i in TMEM
+    // With two dP^T buffers the warpgroups can finish tile i+1 before the MMA
+    // thread has seen their arrivals for tile i, so P^T and dS^T readiness
+    // alternate between two barriers each (a parity wait cannot tell two
+    // completed phases of one barrier apart); with one buffer, one each.
     uint64_t *dp_full = s_full + 1;           // MMA -> WGs: dP^T_i in TMEM (one per dP^T buffer)
     uint64_t *s_free = dp_full + 2;           // WGs -> MMA: S^T_i read
-    uint64_t *p_ready = s_free + 1;           // WGs -> MMA: P^T_i in TMEM
-    uint64_t *ds_ready = p_ready + 1;         // WGs -> MMA: dS^T_i in TMEM
-    uint64_t *drain = ds_ready + 1;
-    static_assert(7 <= Lay::MAX_HANDOFF, "barrier count");
+    uint64_t *p_ready = s_free + 1;           // [2] WGs -> MMA: P^T_i in TMEM
+    uint64_t *ds_ready = p_ready + 2;         // [2] WGs -> MMA: dS^T_i in TMEM
+    uint64_t *drain = ds_ready + 2;
+    static_assert(9 <= Lay::MAX_HANDOFF, "barrier count");
+    // barrier index and phase parity of tile i's P^T / dS^T readiness
+    auto rdy = [](int i) { return Lay::DP2 ? (i & 1) : 0; };
+    auto rdy_par = [](int i) { return static_cast<uint32_t>(Lay::DP2 ? ((i >> 1) & 1) : (i & 1)); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -590,8 +597,10 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
         mbar_init(&dp_full[0], 1);
         mbar_init(&dp_full[1], 1);
         mbar_init(s_free, BwdSigma<D>::kArrivals);
-        mbar_init(p_ready, BwdSigma<D>::kArrivals);
-        mbar_init(ds_ready, BwdSigma<D>::kArrivals);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&p_ready[b], BwdSigma<D>::kArrivals);
+            mbar_init(&ds_ready[b], BwdSigma<D>::kArrivals);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -701,12 +710,12 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
                         mma_commit_w(&dp_full[(i + 1) & 1]);
                     }
                 }
-                if (!(ok = wait(p_ready, i & 1))) break;
+                if (!(ok = wait(&p_ready[rdy(i)], rdy_par(i)))) break;
                 if (lane == 0) trace(1, i, 1);
                 tc_fence_after();
                 issue_acc(Lay::COL_ACC0, dpcol(i), doslot(i), i == 0);          // dV += P^T dO_i
                 mma_commit_w(&y_empty[i % SY]);                                 // dO_i: dP^T_i, dV_i done
-                if (!(ok = wait(ds_ready, i & 1))) break;
+                if (!(ok = wait(&ds_ready[rdy(i)], rdy_par(i)))) break;
                 if (lane == 0) trace(1, i, 2);
                 tc_fence_after();
                 issue_acc(Lay::COL_ACC1, dpcol(i) + SG::kPacked, qslot(i), i == 0);  // dK += dS^T Q_i
@@ -787,13 +796,13 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(p_ready);
+                    mbar_arrive(&p_ready[rdy(i)]);
                     if (qvalid < 128) mask_packed(ds, SG::kCols * w, qvalid);
                     // dS^T over the other half, read in chunk 1
                     tmem_st16(tD + SG::kPacked, ds);
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(ds_ready);
+                    mbar_arrive(&ds_ready[rdy(i)]);
                     if (quarter == 0) trace(2 + (w & 1), i, 4);
                 }
             } else {
@@ -840,7 +849,7 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
                         }
                         tmem_wait_st();
                         tc_fence_before();
-                        mbar_arrive(p_ready);
+                        mbar_arrive(&p_ready[rdy(i)]);
                     }
                     {
                         // the other kPacked dP^T columns, then dS^T over them
@@ -857,7 +866,7 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
                     tmem_st_cols(tD + SG::kPacked, ds);
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(ds_ready);
+                    mbar_arrive(&ds_ready[rdy(i)]);
                     if (quarter == 0) trace(2 + (w & 1), i, 4);
                 }
             }
