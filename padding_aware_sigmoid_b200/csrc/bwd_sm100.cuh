@@ -66,10 +66,6 @@ struct BwdLayout {
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
     static_assert(COL_ACC1 + D <= TMEM_COLS, "TMEM budget");
-    // dK/dV: where the TMEM has room (D = 64) a second dP^T buffer alternates
-    // with the first between query tiles
-    static constexpr bool DP2 = COL_ACC1 + D + 128 <= TMEM_COLS;
-    static constexpr uint32_t COL_DP1 = DP2 ? COL_ACC1 + D : COL_DP;
     static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
@@ -510,22 +506,16 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
 //   S^T = K Q_i^T, dP^T = V dO_i^T, P^T and dS^T -> TMEM over dP^T,
 //   dV += P^T dO_i, dK += dS^T Q_i.
 // TMEM: [0,128) S^T, [128,256) dP^T, then P^T and dS^T over it,
-// [256,256+D) dV, [256+D,256+2D) dK; at D = 64 a second dP^T buffer in
-// [384,512), the two alternating between query tiles.
+// [256,256+D) dV, [256+D,256+2D) dK.
 //
 // A warpgroup reads its kCols columns of S^T into registers and releases the
-// S^T buffer at once, so S^T_{i+1} is computed while it works on tile i.  It
-// writes P^T (its kCols tile columns packed two per TMEM column) over the first
-// half of its dP^T columns once it has read them, and dS^T over the other half.
-// With one dP^T buffer (D = 128) it evaluates sigma and sigma' while dP^T_i is
-// still being computed, keeping P^T and sigma' in registers, and the MMA order
-// per query tile is S^T_{i+1} (as soon as S^T_i is read), dV_i, dK_i, dP^T_{i+1}
-// (over P^T_i and dS^T_i, read by dV_i and dK_i just before: MMAs from one
-// thread run in issue order).  With two (D = 64) dP^T_{i+1} follows S^T_{i+1}
-// at once, into the buffer of tile i-1 (whose readers dV_{i-1} and dK_{i-1}
-// were issued before), so dP^T_i is ready when the warpgroup starts tile i and
-// it forms P^T, sigma' and dS^T in one pass, 16 tile columns at a time, the
-// MUFU work of one chunk overlapping the packing of the other.
+// S^T buffer at once, so S^T_{i+1} is computed while it evaluates sigma and
+// sigma' for tile i.  It keeps P^T in registers until it has read the first
+// half of its dP^T columns, then writes P^T over them (its kCols tile columns
+// packed two per TMEM column) and dS^T over the other half.  MMA order per query
+// tile: S^T_{i+1} (as soon as S^T_i is read), dV_i, dK_i, dP^T_{i+1} (over P^T_i
+// and dS^T_i, read by dV_i and dK_i just before: MMAs from one thread run in
+// issue order).
 // ============================================================================
 template <int D, int MODE, int SX, int SY>
 __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
@@ -543,19 +533,12 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
     uint64_t *y_full = x_empty + SX;          // dO_i ring
     uint64_t *y_empty = y_full + SY;
     uint64_t *s_full = y_empty + SY;          // MMA -> WGs: S^T_i in TMEM
-    // With two dP^T buffers the warpgroups can finish tile i+1 before the MMA
-    // thread has seen their arrivals for tile i, so P^T and dS^T readiness
-    // alternate between two barriers each (a parity wait cannot tell two
-    // completed phases of one barrier apart); with one buffer, one each.
-    uint64_t *dp_full = s_full + 1;           // MMA -> WGs: dP^T_i in TMEM (one per dP^T buffer)
-    uint64_t *s_free = dp_full + 2;           // WGs -> MMA: S^T_i read
-    uint64_t *p_ready = s_free + 1;           // [2] WGs -> MMA: P^T_i in TMEM
-    uint64_t *ds_ready = p_ready + 2;         // [2] WGs -> MMA: dS^T_i in TMEM
-    uint64_t *drain = ds_ready + 2;
-    static_assert(9 <= Lay::MAX_HANDOFF, "barrier count");
-    // barrier index and phase parity of tile i's P^T / dS^T readiness
-    auto rdy = [](int i) { return Lay::DP2 ? (i & 1) : 0; };
-    auto rdy_par = [](int i) { return static_cast<uint32_t>(Lay::DP2 ? ((i >> 1) & 1) : (i & 1)); };
+    uint64_t *dp_full = s_full + 1;           // MMA -> WGs: dP^T_i in TMEM
+    uint64_t *s_free = dp_full + 1;           // WGs -> MMA: S^T_i read
+    uint64_t *p_ready = s_free + 1;           // WGs -> MMA: P^T_i in TMEM
+    uint64_t *ds_ready = p_ready + 1;         // WGs -> MMA: dS^T_i in TMEM
+    uint64_t *drain = ds_ready + 1;
+    static_assert(6 <= Lay::MAX_HANDOFF, "barrier count");
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::OFF_TMEM);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::OFF_ABORT);
 
@@ -594,13 +577,10 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
             mbar_init(&y_empty[s], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(&dp_full[0], 1);
-        mbar_init(&dp_full[1], 1);
+        mbar_init(dp_full, 1);
         mbar_init(s_free, BwdSigma<D>::kArrivals);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&p_ready[b], BwdSigma<D>::kArrivals);
-            mbar_init(&ds_ready[b], BwdSigma<D>::kArrivals);
-        }
+        mbar_init(p_ready, BwdSigma<D>::kArrivals);
+        mbar_init(ds_ready, BwdSigma<D>::kArrivals);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -687,10 +667,8 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
                 issue_xyT(Lay::COL_S, sK, qslot(0));
                 mma_commit_w(s_full);
                 issue_xyT(Lay::COL_DP, sV, doslot(0));
-                mma_commit_w(&dp_full[0]);
+                mma_commit_w(dp_full);
             }
-            // dP^T buffer of query tile i (two alternate where the TMEM has room)
-            auto dpcol = [&](int i) { return (Lay::DP2 && (i & 1)) ? Lay::COL_DP1 : Lay::COL_DP; };
             for (int i = 0; ok && i < nqt; ++i) {
                 const bool more = i + 1 < nqt;
                 if (more) {
@@ -701,33 +679,25 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
                     tc_fence_after();
                     issue_xyT(Lay::COL_S, sK, qslot(i + 1));
                     mma_commit_w(s_full);
-                    if constexpr (Lay::DP2) {
-                        // dP^T_{i+1} into the other buffer at once: its P^T_{i-1} and
-                        // dS^T_{i-1} were read by dV_{i-1} and dK_{i-1}, issued earlier
-                        if (!(ok = wait(&y_full[(i + 1) % SY], ((i + 1) / SY) & 1))) break;
-                        tc_fence_after();
-                        issue_xyT(dpcol(i + 1), sV, doslot(i + 1));
-                        mma_commit_w(&dp_full[(i + 1) & 1]);
-                    }
                 }
-                if (!(ok = wait(&p_ready[rdy(i)], rdy_par(i)))) break;
+                if (!(ok = wait(p_ready, i & 1))) break;
                 if (lane == 0) trace(1, i, 1);
                 tc_fence_after();
-                issue_acc(Lay::COL_ACC0, dpcol(i), doslot(i), i == 0);          // dV += P^T dO_i
+                issue_acc(Lay::COL_ACC0, Lay::COL_DP, doslot(i), i == 0);       // dV += P^T dO_i
                 mma_commit_w(&y_empty[i % SY]);                                 // dO_i: dP^T_i, dV_i done
-                if (!(ok = wait(&ds_ready[rdy(i)], rdy_par(i)))) break;
+                if (!(ok = wait(ds_ready, i & 1))) break;
                 if (lane == 0) trace(1, i, 2);
                 tc_fence_after();
-                issue_acc(Lay::COL_ACC1, dpcol(i) + SG::kPacked, qslot(i), i == 0);  // dK += dS^T Q_i
+                issue_acc(Lay::COL_ACC1, Lay::COL_DP + SG::kPacked, qslot(i), i == 0);  // dK += dS^T Q_i
                 mma_commit_w(&x_empty[i % SX]);                                 // Q_i: S^T_i, dK_i done
-                if (!Lay::DP2 && more) {
+                if (more) {
                     // dP^T_{i+1} overwrites P^T_i and dS^T_i, read by the two MMAs just
                     // issued (MMAs run in issue order)
                     if (!(ok = wait(&y_full[(i + 1) % SY], ((i + 1) / SY) & 1))) break;
                     if (lane == 0) trace(1, i, 3);
                     tc_fence_after();
                     issue_xyT(Lay::COL_DP, sV, doslot(i + 1));
-                    mma_commit_w(&dp_full[0]);
+                    mma_commit_w(dp_full);
                 }
             }
             mma_commit_w(drain);
@@ -750,125 +720,68 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
         {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             const uint32_t tS = tmem + lane_bits + Lay::COL_S + SG::kCols * w;
-            if constexpr (Lay::DP2) {
-                // dP^T_i was issued right after S^T_i (second dP^T buffer), so
-                // P^T, sigma' and dS^T are formed in one pass, 16 tile columns at a
-                // time: the MUFU work of one chunk overlaps the multiplies and bf16
-                // packing of the other
-                static_assert(SG::kCols == 32, "one pass over 32 columns per warpgroup");
-                for (int i = 0; i < nqt; ++i) {
-                    const int qvalid = nq - i * 128;
-                    if (quarter == 0) trace(2 + (w & 1), i, 0);
-                    ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
-                    if (!ok) break;
-                    if (quarter == 0) trace(2 + (w & 1), i, 1);
-                    tc_fence_after();
+            const uint32_t tD = tmem + lane_bits + Lay::COL_DP + SG::kCols * w;
+            for (int i = 0; i < nqt; ++i) {
+                const int qvalid = nq - i * 128;
+                float2 g[SG::kPacked];
+                uint32_t pk[SG::kPacked];
+                if (quarter == 0) trace(2 + (w & 1), i, 0);
+                ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
+                if (!ok) break;
+                if (quarter == 0) trace(2 + (w & 1), i, 1);
+                tc_fence_after();
+                {
                     uint32_t r[SG::kCols];
                     tmem_ld_cols(tS, r);
                     // S^T_i is in registers: the MMA warp may compute S^T_{i+1} now
                     tc_fence_before();
                     mbar_arrive(s_free);
-                    ok = __all_sync(0xffffffffu, mbar_wait(&dp_full[i & 1], (i >> 1) & 1, wctx));
-                    if (!ok) break;
-                    if (quarter == 0) trace(2 + (w & 1), i, 3);
-                    tc_fence_after();
-                    const uint32_t tD =
-                        tmem + lane_bits + ((i & 1) ? Lay::COL_DP1 : Lay::COL_DP) + SG::kCols * w;
-                    uint32_t ds[SG::kPacked];
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        uint32_t d[16];
-                        tmem_ld16(tD + 16 * ch, d);
-                        uint32_t pk[8];
-#pragma unroll
-                        for (int ii = 0; ii < 8; ++ii) {
-                            const int k = 8 * ch + ii;
-                            float2 pr, g;
-                            sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]), cf),
-                                              pr, g);
-                            pk[ii] = pack_bf16x2(pr.x, pr.y);
-                            const float2 v = mul2(g, f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
-                            ds[k] = pack_bf16x2(v.x, v.y);
-                        }
-                        if (qvalid < 128) mask_packed(pk, SG::kCols * w + 16 * ch, qvalid);
-                        // P^T over dP^T columns [8 ch, 8 ch + 8), read in chunk 0
-                        tmem_st8(tD + 8 * ch, pk);
+                    for (int ii = 0; ii < SG::kPacked; ++ii) {
+                        float2 pr;
+                        sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * ii]), __uint_as_float(r[2 * ii + 1]), cf),
+                                          pr, g[ii]);
+                        pk[ii] = pack_bf16x2(pr.x, pr.y);
                     }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(&p_ready[rdy(i)]);
-                    if (qvalid < 128) mask_packed(ds, SG::kCols * w, qvalid);
-                    // dS^T over the other half, read in chunk 1
-                    tmem_st16(tD + SG::kPacked, ds);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(&ds_ready[rdy(i)]);
-                    if (quarter == 0) trace(2 + (w & 1), i, 4);
                 }
-            } else {
-                const uint32_t tD = tmem + lane_bits + Lay::COL_DP + SG::kCols * w;
-                for (int i = 0; i < nqt; ++i) {
-                    const int qvalid = nq - i * 128;
-                    float2 g[SG::kPacked];
-                    uint32_t pk[SG::kPacked];
-                    if (quarter == 0) trace(2 + (w & 1), i, 0);
-                    ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
-                    if (!ok) break;
-                    if (quarter == 0) trace(2 + (w & 1), i, 1);
-                    tc_fence_after();
-                    {
-                        uint32_t r[SG::kCols];
-                        tmem_ld_cols(tS, r);
-                        // S^T_i is in registers: the MMA warp may compute S^T_{i+1} now
-                        tc_fence_before();
-                        mbar_arrive(s_free);
+                if (qvalid < 128) mask_packed(pk, SG::kCols * w, qvalid);
+                if (quarter == 0) trace(2 + (w & 1), i, 2);
+                ok = __all_sync(0xffffffffu, mbar_wait(dp_full, i & 1, wctx));
+                if (!ok) break;
+                if (quarter == 0) trace(2 + (w & 1), i, 3);
+                tc_fence_after();
+                uint32_t ds[SG::kPacked];
+                {
+                    // the first kPacked of this warpgroup's dP^T columns, then P^T over them
+                    uint32_t d[SG::kPacked];
+                    tmem_ld_cols(tD, d);
+                    tmem_st_cols(tD, pk);
 #pragma unroll
-                        for (int ii = 0; ii < SG::kPacked; ++ii) {
-                            float2 pr;
-                            sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * ii]), __uint_as_float(r[2 * ii + 1]), cf),
-                                              pr, g[ii]);
-                            pk[ii] = pack_bf16x2(pr.x, pr.y);
-                        }
+                    for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
+                        const float2 v = mul2(g[ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
+                        ds[ii] = pack_bf16x2(v.x, v.y);
                     }
-                    if (qvalid < 128) mask_packed(pk, SG::kCols * w, qvalid);
-                    if (quarter == 0) trace(2 + (w & 1), i, 2);
-                    ok = __all_sync(0xffffffffu, mbar_wait(&dp_full[0], i & 1, wctx));
-                    if (!ok) break;
-                    if (quarter == 0) trace(2 + (w & 1), i, 3);
-                    tc_fence_after();
-                    uint32_t ds[SG::kPacked];
-                    {
-                        // the first kPacked of this warpgroup's dP^T columns, then P^T over them
-                        uint32_t d[SG::kPacked];
-                        tmem_ld_cols(tD, d);
-                        tmem_st_cols(tD, pk);
-#pragma unroll
-                        for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
-                            const float2 v = mul2(g[ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
-                            ds[ii] = pack_bf16x2(v.x, v.y);
-                        }
-                        tmem_wait_st();
-                        tc_fence_before();
-                        mbar_arrive(&p_ready[rdy(i)]);
-                    }
-                    {
-                        // the other kPacked dP^T columns, then dS^T over them
-                        uint32_t d[SG::kPacked];
-                        tmem_ld_cols(tD + SG::kPacked, d);
-#pragma unroll
-                        for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
-                            const float2 v = mul2(g[SG::kPacked / 2 + ii],
-                                                  f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
-                            ds[SG::kPacked / 2 + ii] = pack_bf16x2(v.x, v.y);
-                        }
-                    }
-                    if (qvalid < 128) mask_packed(ds, SG::kCols * w, qvalid);
-                    tmem_st_cols(tD + SG::kPacked, ds);
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(&ds_ready[rdy(i)]);
-                    if (quarter == 0) trace(2 + (w & 1), i, 4);
+                    mbar_arrive(p_ready);
                 }
+                {
+                    // the other kPacked dP^T columns, then dS^T over them
+                    uint32_t d[SG::kPacked];
+                    tmem_ld_cols(tD + SG::kPacked, d);
+#pragma unroll
+                    for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
+                        const float2 v = mul2(g[SG::kPacked / 2 + ii],
+                                              f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
+                        ds[SG::kPacked / 2 + ii] = pack_bf16x2(v.x, v.y);
+                    }
+                }
+                if (qvalid < 128) mask_packed(ds, SG::kCols * w, qvalid);
+                tmem_st_cols(tD + SG::kPacked, ds);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(ds_ready);
+                if (quarter == 0) trace(2 + (w & 1), i, 4);
             }
             // every MMA of this CTA has finished once the MMA thread's final commit lands
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
