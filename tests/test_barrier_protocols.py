@@ -1,0 +1,370 @@
+"""Host-side model check of the backward kernels' barrier protocols.
+
+Each role of a block (the two TMA producers, the MMA issuer, the sigma
+warpgroups) is written as the sequence of barrier waits, arrivals, tensor-core
+MMAs, commits, TMA loads and TMEM reads and writes that the kernels in
+bwd_sm100.cuh run.  MMAs and commits complete in issue order at arbitrary
+later times (one tensor pipe per block), and TMA loads land at arbitrary later
+times.  Many random interleavings, with per-run random speeds per role, are
+explored, and each is checked for:
+
+* parity aliasing: an mbarrier parity wait cannot tell phase k from phase
+  k + 2, so a wait that starts when its barrier has already completed two
+  phases past the one it wants blocks for good (the kernel would end in its
+  bounded-wait timeout);
+* miscounted phases: every arrival lands in the phase its sender means (a
+  fast warpgroup's arrival for tile i + 1 must never complete tile i's phase);
+* data flow: every read of a TMEM buffer, ring slot or accumulator, by an MMA
+  when it runs or by a warpgroup when it loads, finds the tile it expects;
+* progress: every role finishes (no deadlock).
+
+The kernels' protocols pass at several ring depths, tile counts and
+warpgroup counts.  Three planted mistakes must be caught: the two-buffer
+dK/dV form with one readiness barrier each for P^T and dS^T (the warpgroups
+can finish tile i + 1 before the MMA thread has waited for tile i), an S MMA
+issued without waiting for the warpgroups to have read the previous S, and a
+P^T readiness arrival sent before P^T is written.
+"""
+import random
+import re
+
+import pytest
+
+
+class ProtocolError(Exception):
+    pass
+
+
+class Barrier:
+    def __init__(self, count):
+        self.count, self.arrived, self.done = count, 0, 0   # done: completed phases
+
+    def arrive(self, who, name, phase):
+        if phase is not None and phase != self.done:
+            raise ProtocolError(f"{who} arrives on {name} for phase {phase}, "
+                                f"but phase {self.done} is open")
+        self.arrived += 1
+        if self.arrived == self.count:
+            self.arrived, self.done = 0, self.done + 1
+
+
+class Model:
+    """Roles are generators of ops:
+    ('wait', bar, phase)                  parity wait for `phase` of `bar`
+    ('arrive', bar, phase)                plain arrival on the open `phase`
+    ('mma', reads, writes)                queued on the pipe; reads/writes are
+                                          lists of (buffer, tile)
+    ('commit', bar, phase)                queued; arrives once earlier MMAs ran
+    ('tma', bar, phase, buffer, tile)     lands later, then arrives
+    ('use', buffer, tile)                 warpgroup reads a buffer now
+    ('write', buffer, tile)               warpgroup writes a buffer now"""
+
+    def __init__(self, barriers, roles, seed):
+        self.bars = {k: Barrier(c) for k, c in barriers.items()}
+        self.roles = roles
+        self.rng = random.Random(seed)
+        self.speed = {name: self.rng.choice((0.05, 0.3, 1.0, 3.0)) for name in roles}
+        self.speed["pipe"] = self.rng.choice((0.1, 1.0, 3.0))
+        self.speed["tma"] = self.rng.choice((0.1, 1.0, 3.0))
+        self.buf = {}
+        self.pipe = []
+        self.tma = []
+
+    def _check(self, who, buffer, tile):
+        got = self.buf.get(buffer)
+        if got != tile:
+            raise ProtocolError(f"{who} reads {buffer} expecting {tile}, finds {got}")
+
+    def run(self, max_steps=500000):
+        gens = dict(self.roles)
+        cur = {name: next(g) for name, g in gens.items()}
+        for _ in range(max_steps):
+            ready = []
+            for name, op in cur.items():
+                if op is None:
+                    continue
+                if op[0] == "wait":
+                    bar = self.bars[op[1]]
+                    if bar.done >= op[2] + 2:
+                        raise ProtocolError(f"{name} waits for phase {op[2]} of {op[1]}, "
+                                            f"which has completed {bar.done} phases")
+                    if bar.done == op[2] + 1:
+                        ready.append(name)
+                else:
+                    ready.append(name)
+            if self.pipe:
+                ready.append("pipe")
+            if self.tma:
+                ready.append("tma")
+            if not ready:
+                if all(op is None for op in cur.values()):
+                    return
+                raise ProtocolError("deadlock: " + "; ".join(
+                    f"{n} at {op}" for n, op in cur.items() if op is not None))
+            ev = self.rng.choices(ready, weights=[self.speed[e] for e in ready])[0]
+            if ev == "pipe":
+                item = self.pipe.pop(0)
+                if item[0] == "mma":
+                    for b, t in item[1]:
+                        self._check("an MMA", b, t)
+                    for b, t in item[2]:
+                        self.buf[b] = t
+                else:
+                    self.bars[item[1]].arrive("a commit", item[1], item[2])
+                continue
+            if ev == "tma":
+                _, bar, phase, b, t = self.tma.pop(self.rng.randrange(len(self.tma)))
+                self.buf[b] = t
+                self.bars[bar].arrive("a TMA load", bar, phase)
+                continue
+            op = cur[ev]
+            kind = op[0]
+            if kind == "arrive":
+                self.bars[op[1]].arrive(ev, op[1], op[2])
+            elif kind in ("mma", "commit"):
+                self.pipe.append(op)
+            elif kind == "tma":
+                self.tma.append(op)
+            elif kind == "use":
+                self._check(ev, op[1], op[2])
+            elif kind == "write":
+                self.buf[op[1]] = op[2]
+            cur[ev] = next(gens[ev], None)
+        raise ProtocolError("step limit")
+
+
+def _ring_producer(n, S, full, empty, ring, tile, resident=()):
+    """ring_load over tiles 0..n-1 into S slots, then ring_drain; `resident`
+    lists (buffer, tile) loads issued first on the res_full barrier."""
+    def g():
+        for b, t in resident:
+            yield ("tma", "res_full", 0, b, t)
+        for j in range(n):
+            if j >= S:
+                yield ("wait", f"{empty}{j % S}", j // S - 1)
+            yield ("tma", f"{full}{j % S}", j // S, f"{ring}{j % S}", f"{tile}{j}")
+        if resident:
+            yield ("wait", "res_full", 0)
+        for j in range(max(n - S, 0), n):
+            yield ("wait", f"{full}{j % S}", j // S)
+    return g()
+
+
+def _ring_barriers(SX, SY):
+    bars = {"res_full": 2, "s_full": 1, "drain": 1}
+    for s in range(SX):
+        bars[f"x_full{s}"] = 1
+        bars[f"x_empty{s}"] = 1
+    for s in range(SY):
+        bars[f"y_full{s}"] = 1
+        bars[f"y_empty{s}"] = 1
+    return bars
+
+
+# ---------------------------------------------------------------- dK/dV kernel
+#
+# One block owns a 128-key tile; Q_i and dO_i stream through rings X and Y.
+# Per query tile i: S^T_i = K Q_i^T and dP^T_i = V dO_i^T into TMEM; each
+# warpgroup w turns its columns of dP^T into P^T (first half, packed bf16)
+# and dS^T (second half); dV += P^T dO_i, dK += dS^T Q_i.
+
+def dkdv_roles(n, SX, SY, NG, mistake=None):
+    two_dp = mistake == "dp2_single_ready"
+    W = range(NG)
+
+    def dpa(i, w):
+        return f"dPa{i & 1 if two_dp else 0}.{w}"
+
+    def dpb(i, w):
+        return f"dPb{i & 1 if two_dp else 0}.{w}"
+
+    def dp_bar(i):
+        return (f"dp_full{i & 1}", i >> 1) if two_dp else ("dp_full0", i)
+
+    def s_mma(i):
+        return ("mma", [("K", "K"), (f"X{i % SX}", f"Q{i}")], [(f"S.{w}", f"S{i}") for w in W])
+
+    def dp_mma(i):
+        return ("mma", [("V", "V"), (f"Y{i % SY}", f"dO{i}")],
+                [(dpa(i, w), f"dP{i}") for w in W] + [(dpb(i, w), f"dP{i}") for w in W])
+
+    def mma():
+        yield ("wait", "res_full", 0)
+        yield ("wait", "x_full0", 0)
+        yield ("wait", "y_full0", 0)
+        yield s_mma(0)
+        yield ("commit", "s_full", 0)
+        yield dp_mma(0)
+        yield ("commit", *dp_bar(0))
+        for i in range(n):
+            more = i + 1 < n
+            if more:
+                yield ("wait", f"x_full{(i + 1) % SX}", (i + 1) // SX)
+                if mistake != "no_s_free_wait":
+                    yield ("wait", "s_free", i)
+                yield s_mma(i + 1)
+                yield ("commit", "s_full", i + 1)
+                if two_dp:
+                    yield ("wait", f"y_full{(i + 1) % SY}", (i + 1) // SY)
+                    yield dp_mma(i + 1)
+                    yield ("commit", *dp_bar(i + 1))
+            yield ("wait", "p_ready", i)
+            yield ("mma", [(dpa(i, w), f"P{i}") for w in W] + [(f"Y{i % SY}", f"dO{i}")] +
+                   ([("dV", f"dV{i - 1}")] if i else []), [("dV", f"dV{i}")])
+            yield ("commit", f"y_empty{i % SY}", i // SY)
+            yield ("wait", "ds_ready", i)
+            yield ("mma", [(dpb(i, w), f"dS{i}") for w in W] + [(f"X{i % SX}", f"Q{i}")] +
+                   ([("dK", f"dK{i - 1}")] if i else []), [("dK", f"dK{i}")])
+            yield ("commit", f"x_empty{i % SX}", i // SX)
+            if more and not two_dp:
+                yield ("wait", f"y_full{(i + 1) % SY}", (i + 1) // SY)
+                yield dp_mma(i + 1)
+                yield ("commit", *dp_bar(i + 1))
+        yield ("commit", "drain", 0)
+        yield ("wait", "drain", 0)
+
+    def sigma(w):
+        for i in range(n):
+            yield ("wait", "s_full", i)
+            yield ("use", f"S.{w}", f"S{i}")
+            yield ("arrive", "s_free", i)
+            yield ("wait", *dp_bar(i))
+            yield ("use", dpa(i, w), f"dP{i}")
+            if mistake == "p_ready_before_write":
+                yield ("arrive", "p_ready", i)
+                yield ("write", dpa(i, w), f"P{i}")
+            else:
+                yield ("write", dpa(i, w), f"P{i}")
+                yield ("arrive", "p_ready", i)
+            yield ("use", dpb(i, w), f"dP{i}")
+            yield ("write", dpb(i, w), f"dS{i}")
+            yield ("arrive", "ds_ready", i)
+        yield ("wait", "drain", 0)
+        acc = "dV" if w < max(NG // 2, 1) else "dK"
+        yield ("use", acc, f"{acc}{n - 1}")
+
+    bars = _ring_barriers(SX, SY)
+    bars.update({"dp_full0": 1, "dp_full1": 1, "s_free": NG, "p_ready": NG, "ds_ready": NG})
+    roles = {"loadQ": _ring_producer(n, SX, "x_full", "x_empty", "X", "Q", (("K", "K"), ("V", "V"))),
+             "loadDO": _ring_producer(n, SY, "y_full", "y_empty", "Y", "dO"),
+             "mma": mma()}
+    roles.update({f"sigma{w}": sigma(w) for w in W})
+    return bars, roles
+
+
+# ---------------------------------------------------------------- dQ kernel
+#
+# One block owns a 128-query tile; K_j and V_j stream through rings X and Y.
+# Per key tile j: S_j = Q K_j^T into one TMEM buffer, dP_j = dO V_j^T into
+# buffer j % 2; each warpgroup writes dS_j (packed bf16) over its dP_j
+# columns; dQ += dS_j K_j.
+
+def dq_roles(n, SX, SY, NG, mistake=None):
+    W = range(NG)
+
+    def s_mma(j):
+        return ("mma", [("Q", "Q"), (f"X{j % SX}", f"K{j}")], [(f"S.{w}", f"S{j}") for w in W])
+
+    def dp_mma(j):
+        return ("mma", [("dO", "dO"), (f"Y{j % SY}", f"V{j}")], [(f"dP{j & 1}.{w}", f"dP{j}") for w in W])
+
+    def mma():
+        yield ("wait", "res_full", 0)
+        yield ("wait", "x_full0", 0)
+        yield ("wait", "y_full0", 0)
+        yield s_mma(0)
+        yield ("commit", "s_full", 0)
+        yield dp_mma(0)
+        yield ("commit", "dp_full0", 0)
+        yield ("commit", "y_empty0", 0)
+        for j in range(n):
+            if j + 1 < n:
+                yield ("wait", f"x_full{(j + 1) % SX}", (j + 1) // SX)
+                if mistake != "no_s_free_wait":
+                    yield ("wait", "s_free", j)
+                yield s_mma(j + 1)
+                yield ("commit", "s_full", j + 1)
+                yield ("wait", f"y_full{(j + 1) % SY}", (j + 1) // SY)
+                yield dp_mma(j + 1)
+                yield ("commit", f"dp_full{(j + 1) & 1}", (j + 1) >> 1)
+                yield ("commit", f"y_empty{(j + 1) % SY}", (j + 1) // SY)
+            yield ("wait", f"ds_ready{j & 1}", j >> 1)
+            yield ("mma", [(f"dP{j & 1}.{w}", f"dS{j}") for w in W] + [(f"X{j % SX}", f"K{j}")] +
+                   ([("dQ", f"dQ{j - 1}")] if j else []), [("dQ", f"dQ{j}")])
+            yield ("commit", f"x_empty{j % SX}", j // SX)
+        yield ("commit", "drain", 0)
+        yield ("wait", "drain", 0)
+
+    def sigma(w):
+        for j in range(n):
+            yield ("wait", "s_full", j)
+            yield ("use", f"S.{w}", f"S{j}")
+            yield ("arrive", "s_free", j)
+            yield ("wait", f"dp_full{j & 1}", j >> 1)
+            yield ("use", f"dP{j & 1}.{w}", f"dP{j}")
+            yield ("write", f"dP{j & 1}.{w}", f"dS{j}")
+            yield ("arrive", f"ds_ready{j & 1}", j >> 1)
+        yield ("wait", "drain", 0)
+        yield ("use", "dQ", f"dQ{n - 1}")
+
+    bars = _ring_barriers(SX, SY)
+    bars.update({"dp_full0": 1, "dp_full1": 1, "s_free": NG, "ds_ready0": NG, "ds_ready1": NG})
+    roles = {"loadK": _ring_producer(n, SX, "x_full", "x_empty", "X", "K", (("Q", "Q"), ("dO", "dO"))),
+             "loadV": _ring_producer(n, SY, "y_full", "y_empty", "Y", "V"),
+             "mma": mma()}
+    roles.update({f"sigma{w}": sigma(w) for w in W})
+    return bars, roles
+
+
+# ring depths (X, Y) and sigma warpgroups of the two head dimensions
+SHAPES = [pytest.param(3, 2, 2, id="D128"), pytest.param(4, 4, 4, id="D64")]
+TILES = [1, 2, 3, 5, 8]
+SEEDS = 150
+
+
+def _explore(make, seeds=SEEDS):
+    for seed in range(seeds):
+        bars, roles = make()
+        Model(bars, roles, seed).run()
+
+
+def _errors(make, seeds=1500):
+    """The distinct errors that `seeds` runs of a (mistaken) protocol raise."""
+    found = []
+    for seed in range(seeds):
+        bars, roles = make()
+        try:
+            Model(bars, roles, seed).run()
+        except ProtocolError as e:
+            found.append(str(e))
+    return found
+
+
+@pytest.mark.parametrize("n", TILES)
+@pytest.mark.parametrize("SX,SY,NG", SHAPES)
+def test_dkdv_protocol(n, SX, SY, NG):
+    _explore(lambda: dkdv_roles(n, SX, SY, NG))
+
+
+@pytest.mark.parametrize("n", TILES)
+@pytest.mark.parametrize("SX,SY,NG", SHAPES)
+def test_dq_protocol(n, SX, SY, NG):
+    _explore(lambda: dq_roles(n, SX, SY, NG))
+
+
+@pytest.mark.parametrize("NG", [1, 2])
+def test_two_dp_buffers_with_one_readiness_barrier_are_caught(NG):
+    errs = _errors(lambda: dkdv_roles(5, 4, 4, NG, mistake="dp2_single_ready"))
+    # the MMA thread finds p_ready two phases ahead of the one it waits for
+    assert any(re.search(r"mma waits for phase \d+ of p_ready, which has completed", e) for e in errs)
+
+
+@pytest.mark.parametrize("roles", [dkdv_roles, dq_roles])
+def test_s_overwritten_before_read_is_caught(roles):
+    errs = _errors(lambda: roles(4, 3, 2, 2, mistake="no_s_free_wait"))
+    assert any(re.search(r"sigma\d reads S\.\d expecting S\d, finds S\d", e) for e in errs)
+
+
+def test_early_p_ready_arrival_is_caught():
+    errs = _errors(lambda: dkdv_roles(3, 3, 2, 2, mistake="p_ready_before_write"))
+    assert any(re.search(r"an MMA reads dPa0\.\d expecting P\d, finds dP\d", e) for e in errs)
