@@ -630,8 +630,8 @@ def our_arm(args, world, rank, local):
 # the device code: every file a kernel is compiled from, including the ring
 # depths and thread counts; host code (argument checks, caches, launches) is not
 # part of it
-DEVICE_SOURCES = ("fwd_sm100.cuh", "fwd_persist_sm100.cuh", "bwd_sm100.cuh", "sm100.cuh",
-                  "sigmoid.cuh")
+DEVICE_SOURCES = ("fwd_sm100.cuh", "fwd_persist_sm100.cuh", "bwd_sm100.cuh", "bwd_persist_sm100.cuh",
+                  "sm100.cuh", "sigmoid.cuh")
 TRAFFIC_KERNELS = {"fwd": "fwd_tiles_kernel", "bwd_dq": "bwd_dq_kernel",
                    "bwd_dkdv": "bwd_dkdv_kernel"}
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")

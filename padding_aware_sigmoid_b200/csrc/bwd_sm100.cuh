@@ -36,7 +36,8 @@ struct BwdParams {
     int *status;
     uint64_t timeout_ns;
     const float *bias_z;   // device float[Z], one bias per sample; null: the scalar `bias`
-    float *db_part;        // dQ kernel: one partial of db_z = sum dS per CTA, or null
+    float *db_part;        // dQ kernel: one partial of db_z = sum dS per query tile, or null
+    int Z;                 // samples
 };
 
 // Shared memory: two resident tiles (dq: Q, dO; dkdv: K, V) and two rings of
@@ -175,6 +176,182 @@ __device__ __forceinline__ void mask_packed(uint32_t (&pk)[N], int col0, int val
         const uint32_t lo = c < valid ? 0x0000FFFFu : 0u;
         const uint32_t hi = c + 1 < valid ? 0xFFFF0000u : 0u;
         pk[i] &= (lo | hi);
+    }
+}
+
+// One key tile of a dQ sigma warpgroup (w: the warpgroup, which owns tile
+// columns [kCols w, kCols (w + 1))); `trow` is the TMEM address of this
+// thread's lane.  Reads its columns of S (buffer column col_s) once s_full has
+// completed the phase of parity s_par and releases them (s_free); waits for
+// dP (buffer column dcol, barrier dp_full, parity dp_par); writes
+// dS = sigma'(S) dP, packed bf16, over the first kPacked of its dP columns;
+// then arrives on ds_ready.  kvalid: keys of the tile below n_k (the others
+// give dS = 0); with DB, dbacc adds this row's dS over them.  Returns false
+// when a wait gave up.
+template <int D, int MODE, bool DB>
+__device__ __forceinline__ bool dq_sigma_tile(uint32_t trow, int w, uint32_t col_s, uint32_t dcol,
+                                              uint64_t *s_full, uint32_t s_par, uint64_t *s_free,
+                                              uint64_t *dp_full, uint32_t dp_par, uint64_t *ds_ready,
+                                              const SigmoidCoef &cf, int kvalid, float &dbacc,
+                                              const WaitCtx &wctx, int tstep) {
+    using SG = BwdSigma<D>;
+    const int quarter = warp_id() & 3;
+    if (quarter == 0) trace(2 + (w & 1), tstep, 0);
+    if (!__all_sync(0xffffffffu, mbar_wait(s_full, s_par, wctx))) return false;
+    if (quarter == 0) trace(2 + (w & 1), tstep, 1);
+    tc_fence_after();
+    uint32_t r[SG::kCols];
+    tmem_ld_cols(trow + col_s + SG::kCols * w, r);
+    if (quarter == 0) trace(2 + (w & 1), tstep, 2);
+    tc_fence_before();
+    mbar_arrive(s_free);
+    // sigma'(S) and dS = sigma' dP are formed 32 columns at a time, so that
+    // the MUFU work of one chunk overlaps the multiplies and bf16 packing of
+    // the other.  With two chunks (64 columns per warpgroup) the first chunk's
+    // sigma' is taken before dP is waited for, covering the time dP may still
+    // need.
+    constexpr int kChunks = SG::kCols / 32;
+    constexpr int kPre = kChunks > 1 ? 1 : 0;   // chunks of sigma' before the dP wait
+    float2 gpre[16 * kPre + 1];
+#pragma unroll
+    for (int i = 0; i < 16 * kPre; ++i) {
+        float2 pr;
+        sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf), pr, gpre[i]);
+    }
+    const uint32_t dc = dcol + SG::kCols * w;
+    if (quarter == 0) trace(2 + (w & 1), tstep, 3);
+    if (!__all_sync(0xffffffffu, mbar_wait(dp_full, dp_par, wctx))) return false;
+    if (quarter == 0) trace(2 + (w & 1), tstep, 4);
+    tc_fence_after();
+    float2 dsum = f2(0.0f, 0.0f);   // this row's fp32 dS over keys below n_k
+#pragma unroll
+    for (int ch = 0; ch < kChunks; ++ch) {
+        uint32_t d[32];
+        tmem_ld32(trow + dc + 32 * ch, d);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float2 g;
+            if (ch < kPre) {
+                g = gpre[16 * ch + i];
+            } else {
+                float2 pr;
+                sigma_grad2<MODE>(scale2(__uint_as_float(r[32 * ch + 2 * i]),
+                                         __uint_as_float(r[32 * ch + 2 * i + 1]), cf),
+                                  pr, g);
+            }
+            const float2 ds = mul2(g, f2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
+            pk[i] = pack_bf16x2(ds.x, ds.y);
+            if constexpr (DB) {
+                const int c = SG::kCols * w + 32 * ch + 2 * i;
+                dsum.x += c < kvalid ? ds.x : 0.0f;
+                dsum.y += c + 1 < kvalid ? ds.y : 0.0f;
+            }
+        }
+        if (kvalid < 128) mask_packed(pk, SG::kCols * w + 32 * ch, kvalid);
+        // dS over the first kPacked of this warpgroup's dP columns: chunk ch's
+        // 16 packed columns sit over dP columns this warpgroup has read
+        tmem_st16(trow + dc + 16 * ch, pk);
+    }
+    if (quarter == 0) trace(2 + (w & 1), tstep, 5);
+    if constexpr (DB) dbacc += dsum.x + dsum.y;
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(ds_ready);
+    if (quarter == 0) trace(2 + (w & 1), tstep, 6);
+    return true;
+}
+
+// One query tile of a dK/dV sigma warpgroup (w: the warpgroup, which owns
+// tile columns [kCols w, kCols (w + 1))); tS and tD are the TMEM addresses of
+// its columns of S^T and dP^T in this thread's lane.  S^T, dP^T, P^T and dS^T
+// complete one phase per tile, all of parity `par`.  Reads S^T and releases it
+// (s_free); forms P^T = sigma(S^T) and sigma'; once dP^T is in (dp_full) writes
+// P^T over the first half of its dP^T columns (p_ready), then dS^T =
+// sigma' dP^T over the second half (ds_ready).  qvalid: queries of the tile
+// below n_q (the others give P^T = dS^T = 0).  Returns false when a wait gave up.
+template <int D, int MODE>
+__device__ __forceinline__ bool dkdv_sigma_tile(uint32_t tS, uint32_t tD, int w, uint64_t *s_full,
+                                                uint64_t *s_free, uint64_t *dp_full, uint64_t *p_ready,
+                                                uint64_t *ds_ready, uint32_t par, const SigmoidCoef &cf,
+                                                int qvalid, const WaitCtx &wctx, int tstep) {
+    using SG = BwdSigma<D>;
+    const int quarter = warp_id() & 3;
+    float2 g[SG::kPacked];
+    uint32_t pk[SG::kPacked];
+    if (quarter == 0) trace(2 + (w & 1), tstep, 0);
+    if (!__all_sync(0xffffffffu, mbar_wait(s_full, par, wctx))) return false;
+    if (quarter == 0) trace(2 + (w & 1), tstep, 1);
+    tc_fence_after();
+    {
+        uint32_t r[SG::kCols];
+        tmem_ld_cols(tS, r);
+        // S^T is in registers: the MMA warp may compute the next S^T now
+        tc_fence_before();
+        mbar_arrive(s_free);
+#pragma unroll
+        for (int ii = 0; ii < SG::kPacked; ++ii) {
+            float2 pr;
+            sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * ii]), __uint_as_float(r[2 * ii + 1]), cf), pr, g[ii]);
+            pk[ii] = pack_bf16x2(pr.x, pr.y);
+        }
+    }
+    if (qvalid < 128) mask_packed(pk, SG::kCols * w, qvalid);
+    if (quarter == 0) trace(2 + (w & 1), tstep, 2);
+    if (!__all_sync(0xffffffffu, mbar_wait(dp_full, par, wctx))) return false;
+    if (quarter == 0) trace(2 + (w & 1), tstep, 3);
+    tc_fence_after();
+    uint32_t ds[SG::kPacked];
+    {
+        // the first kPacked of this warpgroup's dP^T columns, then P^T over them
+        uint32_t d[SG::kPacked];
+        tmem_ld_cols(tD, d);
+        tmem_st_cols(tD, pk);
+#pragma unroll
+        for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
+            const float2 v = mul2(g[ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
+            ds[ii] = pack_bf16x2(v.x, v.y);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_ready);
+    }
+    {
+        // the other kPacked dP^T columns, then dS^T over them
+        uint32_t d[SG::kPacked];
+        tmem_ld_cols(tD + SG::kPacked, d);
+#pragma unroll
+        for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
+            const float2 v = mul2(g[SG::kPacked / 2 + ii],
+                                  f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
+            ds[SG::kPacked / 2 + ii] = pack_bf16x2(v.x, v.y);
+        }
+    }
+    if (qvalid < 128) mask_packed(ds, SG::kCols * w, qvalid);
+    tmem_st_cols(tD + SG::kPacked, ds);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(ds_ready);
+    if (quarter == 0) trace(2 + (w & 1), tstep, 4);
+    return true;
+}
+
+// Sum of `v` over the 4 NG sigma warps of the block, in a fixed order (each
+// warp's lanes by a butterfly, then the warps in warp order), written to *dst
+// by warp 4.  Every sigma thread must call it; `red` holds 4 NG floats of
+// shared memory.
+template <int D>
+__device__ __forceinline__ void sigma_block_sum(float v, float *red, float *dst) {
+    using SG = BwdSigma<D>;
+    const int warp = warp_id(), lane = lane_id();
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp - 4] = v;
+    sigma_warps_sync(SG::kArrivals);
+    if (warp == 4 && lane == 0) {
+        float t = 0.0f;
+        for (int u = 0; u < 4 * SG::NG; ++u) t += red[u];
+        *dst = t;
     }
 }
 
@@ -394,73 +571,10 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
         {
             const SigmoidCoef cf = make_coef<MODE>(p.alpha, bias_of(p.bias_z, p.bias, z));
             for (int j = 0; j < nkv; ++j) {
-                if (quarter == 0) trace(2 + (w & 1), j, 0);
-                ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, wctx));
+                ok = dq_sigma_tile<D, MODE, DB>(tmem + lane_bits, w, kColS, j & 1 ? kColDP1 : kColDP0, s_full,
+                                                j & 1, s_free, &dp_full[j & 1], (j >> 1) & 1, &ds_ready[j & 1],
+                                                cf, nk - j * 128, dbacc, wctx, j);
                 if (!ok) break;
-                if (quarter == 0) trace(2 + (w & 1), j, 1);
-                tc_fence_after();
-                uint32_t r[SG::kCols];
-                tmem_ld_cols(tmem + lane_bits + kColS + SG::kCols * w, r);
-                if (quarter == 0) trace(2 + (w & 1), j, 2);
-                tc_fence_before();
-                mbar_arrive(s_free);
-                // sigma'(S_j) and dS_j = sigma' dP_j are formed 32 columns at a
-                // time, so that the MUFU work of one chunk overlaps the multiplies
-                // and bf16 packing of the other.  With two chunks (64 columns per
-                // warpgroup) the first chunk's sigma' is taken before dP_j is
-                // waited for, covering the time dP_j may still need.
-                constexpr int kChunks = SG::kCols / 32;
-                constexpr int kPre = kChunks > 1 ? 1 : 0;   // chunks of sigma' before the dP wait
-                float2 gpre[16 * kPre + 1];
-#pragma unroll
-                for (int i = 0; i < 16 * kPre; ++i) {
-                    float2 pr;
-                    sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), cf), pr,
-                                      gpre[i]);
-                }
-                const uint32_t dcol = (j & 1 ? kColDP1 : kColDP0) + SG::kCols * w;
-                if (quarter == 0) trace(2 + (w & 1), j, 3);
-                ok = __all_sync(0xffffffffu, mbar_wait(&dp_full[j & 1], (j >> 1) & 1, wctx));
-                if (!ok) break;
-                if (quarter == 0) trace(2 + (w & 1), j, 4);
-                tc_fence_after();
-                const int kvalid = nk - j * 128;
-                float2 dsum = f2(0.0f, 0.0f);   // this row's fp32 dS over keys below n_k
-#pragma unroll
-                for (int ch = 0; ch < kChunks; ++ch) {
-                    uint32_t d[32];
-                    tmem_ld32(tmem + lane_bits + dcol + 32 * ch, d);
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float2 g;
-                        if (ch < kPre) {
-                            g = gpre[16 * ch + i];
-                        } else {
-                            float2 pr;
-                            sigma_grad2<MODE>(scale2(__uint_as_float(r[32 * ch + 2 * i]),
-                                                     __uint_as_float(r[32 * ch + 2 * i + 1]), cf),
-                                              pr, g);
-                        }
-                        const float2 ds = mul2(g, f2(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])));
-                        pk[i] = pack_bf16x2(ds.x, ds.y);
-                        if constexpr (DB) {
-                            const int c = SG::kCols * w + 32 * ch + 2 * i;
-                            dsum.x += c < kvalid ? ds.x : 0.0f;
-                            dsum.y += c + 1 < kvalid ? ds.y : 0.0f;
-                        }
-                    }
-                    if (kvalid < 128) mask_packed(pk, SG::kCols * w + 32 * ch, kvalid);
-                    // dS over the first kPacked of this warpgroup's dP columns: chunk
-                    // ch's 16 packed columns sit over dP columns this warpgroup has read
-                    tmem_st16(tmem + lane_bits + dcol + 16 * ch, pk);
-                }
-                if (quarter == 0) trace(2 + (w & 1), j, 5);
-                if constexpr (DB) dbacc += dsum.x + dsum.y;
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&ds_ready[j & 1]);
-                if (quarter == 0) trace(2 + (w & 1), j, 6);
             }
             // every MMA of this CTA has finished once the MMA thread's final commit lands
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));
@@ -474,19 +588,9 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
             }
         }
         if constexpr (DB) {
-            // one partial per CTA, summed in a fixed order: warp sums, then the
-            // 4 NG warps' sums in warp order (rows at or beyond n_q add nothing)
-            float v = row < nq ? dbacc : 0.0f;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            float *red = reinterpret_cast<float *>(smem + Lay::OFF_RED);
-            if (lane == 0) red[warp - 4] = v;
-            sigma_warps_sync(SG::kArrivals);
-            if (warp == 4 && lane == 0) {
-                float t = 0.0f;
-                for (int u = 0; u < 4 * SG::NG; ++u) t += red[u];
-                p.db_part[(static_cast<size_t>(z) * p.H + h) * gridDim.x + qtile] = t;
-            }
+            // one partial per CTA (rows at or beyond n_q add nothing)
+            sigma_block_sum<D>(row < nq ? dbacc : 0.0f, reinterpret_cast<float *>(smem + Lay::OFF_RED),
+                               &p.db_part[(static_cast<size_t>(z) * p.H + h) * gridDim.x + qtile]);
         }
     }
 
@@ -722,66 +826,9 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
             const uint32_t tS = tmem + lane_bits + Lay::COL_S + SG::kCols * w;
             const uint32_t tD = tmem + lane_bits + Lay::COL_DP + SG::kCols * w;
             for (int i = 0; i < nqt; ++i) {
-                const int qvalid = nq - i * 128;
-                float2 g[SG::kPacked];
-                uint32_t pk[SG::kPacked];
-                if (quarter == 0) trace(2 + (w & 1), i, 0);
-                ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, wctx));
+                ok = dkdv_sigma_tile<D, MODE>(tS, tD, w, s_full, s_free, dp_full, p_ready, ds_ready, i & 1, cf,
+                                              nq - i * 128, wctx, i);
                 if (!ok) break;
-                if (quarter == 0) trace(2 + (w & 1), i, 1);
-                tc_fence_after();
-                {
-                    uint32_t r[SG::kCols];
-                    tmem_ld_cols(tS, r);
-                    // S^T_i is in registers: the MMA warp may compute S^T_{i+1} now
-                    tc_fence_before();
-                    mbar_arrive(s_free);
-#pragma unroll
-                    for (int ii = 0; ii < SG::kPacked; ++ii) {
-                        float2 pr;
-                        sigma_grad2<MODE>(scale2(__uint_as_float(r[2 * ii]), __uint_as_float(r[2 * ii + 1]), cf),
-                                          pr, g[ii]);
-                        pk[ii] = pack_bf16x2(pr.x, pr.y);
-                    }
-                }
-                if (qvalid < 128) mask_packed(pk, SG::kCols * w, qvalid);
-                if (quarter == 0) trace(2 + (w & 1), i, 2);
-                ok = __all_sync(0xffffffffu, mbar_wait(dp_full, i & 1, wctx));
-                if (!ok) break;
-                if (quarter == 0) trace(2 + (w & 1), i, 3);
-                tc_fence_after();
-                uint32_t ds[SG::kPacked];
-                {
-                    // the first kPacked of this warpgroup's dP^T columns, then P^T over them
-                    uint32_t d[SG::kPacked];
-                    tmem_ld_cols(tD, d);
-                    tmem_st_cols(tD, pk);
-#pragma unroll
-                    for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
-                        const float2 v = mul2(g[ii], f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
-                        ds[ii] = pack_bf16x2(v.x, v.y);
-                    }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(p_ready);
-                }
-                {
-                    // the other kPacked dP^T columns, then dS^T over them
-                    uint32_t d[SG::kPacked];
-                    tmem_ld_cols(tD + SG::kPacked, d);
-#pragma unroll
-                    for (int ii = 0; ii < SG::kPacked / 2; ++ii) {
-                        const float2 v = mul2(g[SG::kPacked / 2 + ii],
-                                              f2(__uint_as_float(d[2 * ii]), __uint_as_float(d[2 * ii + 1])));
-                        ds[SG::kPacked / 2 + ii] = pack_bf16x2(v.x, v.y);
-                    }
-                }
-                if (qvalid < 128) mask_packed(ds, SG::kCols * w, qvalid);
-                tmem_st_cols(tD + SG::kPacked, ds);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(ds_ready);
-                if (quarter == 0) trace(2 + (w & 1), i, 4);
             }
             // every MMA of this CTA has finished once the MMA thread's final commit lands
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, wctx));

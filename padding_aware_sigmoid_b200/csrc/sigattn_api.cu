@@ -12,6 +12,7 @@
 #include <unordered_set>
 
 #include "../../include/sigattn.h"
+#include "bwd_persist_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "fp32_simt.cuh"
 #include "fwd_persist_sm100.cuh"
@@ -306,27 +307,54 @@ sigattn_status fwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
 
 enum BwdParts : int { kPartDq = 1, kPartDkdv = 2 };
 
+// Head dimension 128: one CTA per tile (bwd_sm100.cuh).  Head dimension 64:
+// one CTA per SM, or per tile when there are fewer, each walking its share of
+// the tiles with work while an idle warp zero-fills the rest
+// (bwd_persist_sm100.cuh): the pages' short, ragged batches at 64 leave most
+// tiles in padding, and a CTA launched per padded tile held its SM for longer
+// than the zeros take to write.
 template <int D, int MODE>
 sigattn_status bwd_bf16(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                         const CUtensorMap &mdo, const BwdParams &p, int Z, int Lq, int Lk,
-                        int H, int parts, cudaStream_t st) {
-    dim3 grid((Lq + 127) / 128, H, Z);      // dQ: one CTA per query tile
-    dim3 grid_kv((Lk + 127) / 128, H, Z);   // dK/dV: one CTA per key tile
-    constexpr int SX = BwdStages<D>::X, SY = BwdStages<D>::Y;
-    constexpr size_t smem = BwdLayout<D, SX, SY>::SMEM_ALLOC;
-    if (parts & kPartDq) {
-        sigattn_status s =
-            p.db_part != nullptr
-                ? launch(bwd_dq_kernel<D, MODE, SX, SY, true>, grid, dim3(BwdSigma<D>::kThreads), smem, st, mq, mk,
-                         mv, mdo, p)
-                : launch(bwd_dq_kernel<D, MODE, SX, SY, false>, grid, dim3(BwdSigma<D>::kThreads), smem, st, mq, mk,
-                         mv, mdo, p);
-        if (s != SIGATTN_OK) return s;
+                        int H, int parts, int sms, cudaStream_t st) {
+    if constexpr (D == 64) {
+        using Lay = BwdPersistLayout<D>;
+        auto grid_of = [&](int L) {
+            const int64_t tiles = static_cast<int64_t>(Z) * H * ((L + 127) / 128);
+            return dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(sms, tiles))));
+        };
+        if (parts & kPartDq) {
+            sigattn_status s =
+                p.db_part != nullptr
+                    ? launch(bwd_dq_persistent_kernel<D, MODE, true>, grid_of(Lq), dim3(BwdSigma<D>::kThreads),
+                             Lay::SMEM_ALLOC, st, mq, mk, mv, mdo, p)
+                    : launch(bwd_dq_persistent_kernel<D, MODE, false>, grid_of(Lq), dim3(BwdSigma<D>::kThreads),
+                             Lay::SMEM_ALLOC, st, mq, mk, mv, mdo, p);
+            if (s != SIGATTN_OK) return s;
+        }
+        if (parts & kPartDkdv)
+            return launch(bwd_dkdv_persistent_kernel<D, MODE>, grid_of(Lk), dim3(BwdSigma<D>::kThreads),
+                          Lay::SMEM_ALLOC, st, mq, mk, mv, mdo, p);
+        return SIGATTN_OK;
+    } else {
+        dim3 grid((Lq + 127) / 128, H, Z);      // dQ: one CTA per query tile
+        dim3 grid_kv((Lk + 127) / 128, H, Z);   // dK/dV: one CTA per key tile
+        constexpr int SX = BwdStages<D>::X, SY = BwdStages<D>::Y;
+        constexpr size_t smem = BwdLayout<D, SX, SY>::SMEM_ALLOC;
+        if (parts & kPartDq) {
+            sigattn_status s =
+                p.db_part != nullptr
+                    ? launch(bwd_dq_kernel<D, MODE, SX, SY, true>, grid, dim3(BwdSigma<D>::kThreads), smem, st,
+                             mq, mk, mv, mdo, p)
+                    : launch(bwd_dq_kernel<D, MODE, SX, SY, false>, grid, dim3(BwdSigma<D>::kThreads), smem, st,
+                             mq, mk, mv, mdo, p);
+            if (s != SIGATTN_OK) return s;
+        }
+        if (parts & kPartDkdv)
+            return launch(bwd_dkdv_kernel<D, MODE, SX, SY>, grid_kv, dim3(BwdSigma<D>::kThreads), smem, st, mq,
+                          mk, mv, mdo, p);
+        return SIGATTN_OK;
     }
-    if (parts & kPartDkdv)
-        return launch(bwd_dkdv_kernel<D, MODE, SX, SY>, grid_kv, dim3(BwdSigma<D>::kThreads), smem, st, mq, mk, mv,
-                      mdo, p);
-    return SIGATTN_OK;
 }
 
 // Partials of db per sample: one per dQ CTA (bf16) or per query row (fp32).
@@ -395,14 +423,14 @@ sigattn_status bwd_impl(const void *q, const void *k, const void *v, const void 
     if ((s = encode_bf16_map(&mdo, dout, Z, Lq, H, D)) != SIGATTN_OK) return s;
     BwdParams p{static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
                 static_cast<__nv_bfloat16 *>(dv), seqlens_q, seqlens_k, Lq, Lk, H, alpha, bias, status,
-                g_timeout_ns.load(), bias_z, db_part};
-    const int mode = g_sigmoid_mode.load();
+                g_timeout_ns.load(), bias_z, db_part, Z};
+    const int mode = g_sigmoid_mode.load(), sms = g_sm_count[dev];
     if (D == 128)
-        s = mode == kSigmoidTanh ? bwd_bf16<128, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, st)
-                                 : bwd_bf16<128, kSigmoidExp>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, st);
+        s = mode == kSigmoidTanh ? bwd_bf16<128, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, sms, st)
+                                 : bwd_bf16<128, kSigmoidExp>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, sms, st);
     else
-        s = mode == kSigmoidTanh ? bwd_bf16<64, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, st)
-                                 : bwd_bf16<64, kSigmoidExp>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, st);
+        s = mode == kSigmoidTanh ? bwd_bf16<64, kSigmoidTanh>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, sms, st)
+                                 : bwd_bf16<64, kSigmoidExp>(mq, mk, mv, mdo, p, Z, Lq, Lk, H, parts, sms, st);
     if (s != SIGATTN_OK || !dbias) return s;
     return launch(dbias_reduce_kernel, dim3(Z), dim3(256), 0, st, static_cast<const float *>(db_part),
                   dbias_partials_per_sample(Lq, H, dtype), dbias);

@@ -368,3 +368,222 @@ def test_s_overwritten_before_read_is_caught(roles):
 def test_early_p_ready_arrival_is_caught():
     errs = _errors(lambda: dkdv_roles(3, 3, 2, 2, mistake="p_ready_before_write"))
     assert any(re.search(r"an MMA reads dPa0\.\d expecting P\d, finds dP\d", e) for e in errs)
+
+
+# ---------------------------------------------------------------- persistent forms
+#
+# One block per SM walks a list of items (tiles with work); an item of n units
+# is one tile's loop above.  The units of all the block's items form one
+# stream: ring slots and hand-off phases run on across items, the resident
+# tiles (dQ: Q, dO; dK/dV: K, V) of consecutive items alternate between NR
+# shared-memory slots (res_full / res_empty), and the MMA thread commits
+# acc_full after an item's last unit, after which the warpgroups read the
+# item's accumulators.  The next item's first accumulating MMA overwrites
+# them only after every warpgroup's next readiness arrival, which comes after
+# those reads.
+
+def _units(items):
+    return [(k, j) for k, n in enumerate(items) for j in range(n)]
+
+
+def _persistent_producer(items, S, full, empty, ring, tile, NR=None, mistake=None):
+    def g():
+        q = 0
+        for k, n in enumerate(items):
+            if NR is not None:
+                rs = k % NR
+                if k >= NR and mistake != "no_res_empty_wait":
+                    yield ("wait", f"res_empty{rs}", k // NR - 1)
+                yield ("tma", f"res_full{rs}", k // NR, f"Res{rs}", f"R{k}")
+            for j in range(n):
+                if q >= S:
+                    yield ("wait", f"{empty}{q % S}", q // S - 1)
+                yield ("tma", f"{full}{q % S}", q // S, f"{ring}{q % S}", f"{tile}{k}.{j}")
+                q += 1
+        if NR is not None:
+            for k in range(max(len(items) - NR, 0), len(items)):
+                yield ("wait", f"res_full{k % NR}", k // NR)
+        for qq in range(max(q - S, 0), q):
+            yield ("wait", f"{full}{qq % S}", qq // S)
+    return g()
+
+
+def _persistent_barriers(SX, SY, NR):
+    bars = _ring_barriers(SX, SY)
+    del bars["res_full"]
+    bars["acc_full"] = 1
+    for r in range(NR):
+        bars[f"res_full{r}"] = 1
+        bars[f"res_empty{r}"] = 1
+    return bars
+
+
+def dq_persistent_roles(items, SX, SY, NG, NR=2, mistake=None):
+    W = range(NG)
+    units = _units(items)
+    U = len(units)
+
+    def s_mma(u):
+        k, j = units[u]
+        return ("mma", [(f"Res{k % NR}", f"R{k}"), (f"X{u % SX}", f"K{k}.{j}")],
+                [(f"S.{w}", f"S{u}") for w in W])
+
+    def dp_mma(u):
+        k, j = units[u]
+        return ("mma", [(f"Res{k % NR}", f"R{k}"), (f"Y{u % SY}", f"V{k}.{j}")],
+                [(f"dP{u & 1}.{w}", f"dP{u}") for w in W])
+
+    def mma():
+        yield ("wait", "res_full0", 0)
+        yield ("wait", "x_full0", 0)
+        yield ("wait", "y_full0", 0)
+        yield s_mma(0)
+        yield ("commit", "s_full", 0)
+        yield dp_mma(0)
+        yield ("commit", "dp_full0", 0)
+        yield ("commit", "y_empty0", 0)
+        for u in range(U):
+            k, j = units[u]
+            if u + 1 < U:
+                k2, j2 = units[u + 1]
+                if j2 == 0:
+                    yield ("wait", f"res_full{k2 % NR}", k2 // NR)
+                yield ("wait", f"x_full{(u + 1) % SX}", (u + 1) // SX)
+                yield ("wait", "s_free", u)
+                yield s_mma(u + 1)
+                yield ("commit", "s_full", u + 1)
+                yield ("wait", f"y_full{(u + 1) % SY}", (u + 1) // SY)
+                yield dp_mma(u + 1)
+                yield ("commit", f"dp_full{(u + 1) & 1}", (u + 1) >> 1)
+                yield ("commit", f"y_empty{(u + 1) % SY}", (u + 1) // SY)
+            yield ("wait", f"ds_ready{u & 1}", u >> 1)
+            yield ("mma", [(f"dP{u & 1}.{w}", f"dS{u}") for w in W] + [(f"X{u % SX}", f"K{k}.{j}")] +
+                   ([("dQ", f"dQ{k}.{j - 1}")] if j else []), [("dQ", f"dQ{k}.{j}")])
+            yield ("commit", f"x_empty{u % SX}", u // SX)
+            if j == items[k] - 1:
+                yield ("commit", f"res_empty{k % NR}", k // NR)
+                yield ("commit", "acc_full", k)
+        yield ("commit", "drain", 0)
+        yield ("wait", "drain", 0)
+
+    def sigma(w):
+        for u in range(U):
+            k, j = units[u]
+            yield ("wait", "s_full", u)
+            yield ("use", f"S.{w}", f"S{u}")
+            yield ("arrive", "s_free", u)
+            yield ("wait", f"dp_full{u & 1}", u >> 1)
+            yield ("use", f"dP{u & 1}.{w}", f"dP{u}")
+            yield ("write", f"dP{u & 1}.{w}", f"dS{u}")
+            yield ("arrive", f"ds_ready{u & 1}", u >> 1)
+            if j == items[k] - 1:
+                yield ("wait", "acc_full", k)
+                yield ("use", "dQ", f"dQ{k}.{j}")
+
+    bars = _persistent_barriers(SX, SY, NR)
+    bars.update({"dp_full0": 1, "dp_full1": 1, "s_free": NG, "ds_ready0": NG, "ds_ready1": NG})
+    roles = {"loadK": _persistent_producer(items, SX, "x_full", "x_empty", "X", "K", NR, mistake),
+             "loadV": _persistent_producer(items, SY, "y_full", "y_empty", "Y", "V"),
+             "mma": mma()}
+    roles.update({f"sigma{w}": sigma(w) for w in W})
+    return bars, roles
+
+
+def dkdv_persistent_roles(items, SX, SY, NG, NR=2, mistake=None):
+    W = range(NG)
+    units = _units(items)
+    U = len(units)
+
+    def s_mma(u):
+        k, i = units[u]
+        return ("mma", [(f"Res{k % NR}", f"R{k}"), (f"X{u % SX}", f"Q{k}.{i}")],
+                [(f"S.{w}", f"S{u}") for w in W])
+
+    def dp_mma(u):
+        k, i = units[u]
+        return ("mma", [(f"Res{k % NR}", f"R{k}"), (f"Y{u % SY}", f"dO{k}.{i}")],
+                [(f"dPa.{w}", f"dP{u}") for w in W] + [(f"dPb.{w}", f"dP{u}") for w in W])
+
+    def mma():
+        yield ("wait", "res_full0", 0)
+        yield ("wait", "x_full0", 0)
+        yield ("wait", "y_full0", 0)
+        yield s_mma(0)
+        yield ("commit", "s_full", 0)
+        yield dp_mma(0)
+        yield ("commit", "dp_full", 0)
+        for u in range(U):
+            k, i = units[u]
+            more = u + 1 < U
+            if more:
+                k2, i2 = units[u + 1]
+                if i2 == 0:
+                    yield ("wait", f"res_full{k2 % NR}", k2 // NR)
+                yield ("wait", f"x_full{(u + 1) % SX}", (u + 1) // SX)
+                yield ("wait", "s_free", u)
+                yield s_mma(u + 1)
+                yield ("commit", "s_full", u + 1)
+            yield ("wait", "p_ready", u)
+            yield ("mma", [(f"dPa.{w}", f"P{u}") for w in W] + [(f"Y{u % SY}", f"dO{k}.{i}")] +
+                   ([("dV", f"dV{k}.{i - 1}")] if i else []), [("dV", f"dV{k}.{i}")])
+            yield ("commit", f"y_empty{u % SY}", u // SY)
+            yield ("wait", "ds_ready", u)
+            yield ("mma", [(f"dPb.{w}", f"dS{u}") for w in W] + [(f"X{u % SX}", f"Q{k}.{i}")] +
+                   ([("dK", f"dK{k}.{i - 1}")] if i else []), [("dK", f"dK{k}.{i}")])
+            yield ("commit", f"x_empty{u % SX}", u // SX)
+            if i == items[k] - 1:
+                yield ("commit", f"res_empty{k % NR}", k // NR)
+                yield ("commit", "acc_full", k)
+            if more:
+                yield ("wait", f"y_full{(u + 1) % SY}", (u + 1) // SY)
+                yield dp_mma(u + 1)
+                yield ("commit", "dp_full", u + 1)
+        yield ("commit", "drain", 0)
+        yield ("wait", "drain", 0)
+
+    def sigma(w):
+        acc = "dV" if w < max(NG // 2, 1) else "dK"
+        for u in range(U):
+            k, i = units[u]
+            yield ("wait", "s_full", u)
+            yield ("use", f"S.{w}", f"S{u}")
+            yield ("arrive", "s_free", u)
+            yield ("wait", "dp_full", u)
+            yield ("use", f"dPa.{w}", f"dP{u}")
+            yield ("write", f"dPa.{w}", f"P{u}")
+            yield ("arrive", "p_ready", u)
+            yield ("use", f"dPb.{w}", f"dP{u}")
+            yield ("write", f"dPb.{w}", f"dS{u}")
+            yield ("arrive", "ds_ready", u)
+            if i == items[k] - 1:
+                yield ("wait", "acc_full", k)
+                yield ("use", acc, f"{acc}{k}.{i}")
+
+    bars = _persistent_barriers(SX, SY, NR)
+    bars.update({"dp_full": 1, "s_free": NG, "p_ready": NG, "ds_ready": NG})
+    roles = {"loadQ": _persistent_producer(items, SX, "x_full", "x_empty", "X", "Q", NR, mistake),
+             "loadDO": _persistent_producer(items, SY, "y_full", "y_empty", "Y", "dO"),
+             "mma": mma()}
+    roles.update({f"sigma{w}": sigma(w) for w in W})
+    return bars, roles
+
+
+ITEM_LISTS = [[1], [3], [1, 1, 1], [3, 1, 2], [1, 4, 1, 1, 2], [5, 5], [2, 1, 1, 1, 1, 3]]
+
+
+@pytest.mark.parametrize("items", ITEM_LISTS, ids=lambda it: "-".join(map(str, it)))
+@pytest.mark.parametrize("SX,SY,NG", SHAPES)
+def test_dq_persistent_protocol(items, SX, SY, NG):
+    _explore(lambda: dq_persistent_roles(items, SX, SY, NG), 100)
+
+
+@pytest.mark.parametrize("items", ITEM_LISTS, ids=lambda it: "-".join(map(str, it)))
+@pytest.mark.parametrize("SX,SY,NG", SHAPES)
+def test_dkdv_persistent_protocol(items, SX, SY, NG):
+    _explore(lambda: dkdv_persistent_roles(items, SX, SY, NG), 100)
+
+
+@pytest.mark.parametrize("roles", [dq_persistent_roles, dkdv_persistent_roles])
+def test_resident_slot_reused_too_early_is_caught(roles):
+    errs = _errors(lambda: roles([1, 1, 1, 2], 4, 4, 4, mistake="no_res_empty_wait"), 800)
+    assert any(re.search(r"reads Res\d expecting R\d, finds R\d", e) for e in errs)

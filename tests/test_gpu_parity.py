@@ -354,11 +354,12 @@ def test_random_shapes_full(seed):
 
 
 @pytest.mark.parametrize("Z,H,L", [(12, 24, 768), (100, 4, 1024)])
-def test_persistent_forward_many_items_per_block(Z, H, L):
-    """Head dimension 64 runs one persistent block per SM: with 12 samples the
-    blocks walk several length-ranked items each (one- and two-tile items
-    mixed), with 100 samples they walk the index-ordered grid and skip items
-    without work.  Every output row against the oracle."""
+def test_persistent_many_items_per_block(Z, H, L):
+    """Head dimension 64 runs the forward and both backward passes as one
+    persistent block per SM: with 12 samples the blocks walk several
+    length-ranked items each (one- and two-tile items mixed in the forward),
+    with 100 samples they walk the index-ordered grid and skip tiles without
+    work, which an idle warp zero-fills.  Every output row against the oracle."""
     dev = _dev()
     g = np.random.default_rng(Z + L)
     nq = g.integers(0, L + 1, size=Z)
