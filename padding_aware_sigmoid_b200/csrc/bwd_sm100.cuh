@@ -207,11 +207,11 @@ __device__ __forceinline__ bool dq_sigma_tile(uint32_t trow, int w, uint32_t col
     mbar_arrive(s_free);
     // sigma'(S) and dS = sigma' dP are formed 32 columns at a time, so that
     // the MUFU work of one chunk overlaps the multiplies and bf16 packing of
-    // the other.  With two chunks (64 columns per warpgroup) the first chunk's
-    // sigma' is taken before dP is waited for, covering the time dP may still
-    // need.
+    // the other.  The first chunk's sigma' (all of it with one chunk of 32
+    // columns, at D = 64) is taken before dP is waited for, covering the time
+    // dP may still need.
     constexpr int kChunks = SG::kCols / 32;
-    constexpr int kPre = kChunks > 1 ? 1 : 0;   // chunks of sigma' before the dP wait
+    constexpr int kPre = 1;   // chunks of sigma' before the dP wait
     float2 gpre[16 * kPre + 1];
 #pragma unroll
     for (int i = 0; i < 16 * kPre; ++i) {
