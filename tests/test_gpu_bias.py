@@ -115,6 +115,23 @@ def test_bias_small_full(Z, L, H, D, nq, nk, mode):
     _check_full(q, k, v, do, nq, nk, alpha, bz, outs, "bf16", DB_TOL[mode])
 
 
+@pytest.mark.parametrize("Z", [12, 70])
+def test_dbias_persistent_many_tiles(Z):
+    """At D = 64 the backward blocks walk the tiles with work (length-ranked up to
+    64 samples, index order above) and an idle warp writes the rows and the db
+    partials of the tiles without work: many tiles per block, empty samples,
+    every output row and db per sample against the oracle."""
+    dev = _dev()
+    g = np.random.default_rng(Z)
+    L, H = (1024, 2) if Z < 64 else (384, 1)   # 192 and 210 tiles for 148 blocks
+    nq = g.integers(0, L + 1, size=Z)
+    nk = g.integers(0, L + 1, size=Z)
+    nq[::9], nk[1::11], nq[2], nk[2] = 0, 0, L, L
+    q, k, v, do, nq, nk, bz = _inputs(Z, L, H, 64, nq, nk, seed=3300 + Z)
+    outs = _run(q, k, v, do, nq, nk, 1.0 / 8.0, bz, dev)
+    _check_full(q, k, v, do, nq, nk, 1.0 / 8.0, bz, outs, "bf16", DB_TOL["tanh"])
+
+
 def test_bias_fp32_full():
     dev = _dev()
     q, k, v, do, nq, nk, bz = _inputs(2, 300, 2, 128, (300, 129), (45, 300), seed=3100,
