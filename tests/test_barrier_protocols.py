@@ -1,9 +1,10 @@
-"""Host-side model check of the backward kernels' barrier protocols.
+"""Host-side model check of the kernels' barrier protocols: the backward
+tile kernels (bwd_sm100.cuh), the persistent backward (bwd_persist_sm100.cuh)
+and the persistent forward (fwd_persist_sm100.cuh).
 
-Each role of a block (the two TMA producers, the MMA issuer, the sigma
+Each role of a block (the TMA producers, the MMA issuer, the sigma
 warpgroups) is written as the sequence of barrier waits, arrivals, tensor-core
-MMAs, commits, TMA loads and TMEM reads and writes that the kernels in
-bwd_sm100.cuh run.  MMAs and commits complete in issue order at arbitrary
+MMAs, commits, TMA loads and TMEM reads and writes that the kernels run.  MMAs and commits complete in issue order at arbitrary
 later times (one tensor pipe per block), and TMA loads land at arbitrary later
 times.  Many random interleavings, with per-run random speeds per role, are
 explored, and each is checked for:
@@ -18,12 +19,15 @@ explored, and each is checked for:
   when it runs or by a warpgroup when it loads, finds the tile it expects;
 * progress: every role finishes (no deadlock).
 
-The kernels' protocols pass at several ring depths, tile counts and
-warpgroup counts.  Three planted mistakes must be caught: the two-buffer
-dK/dV form with one readiness barrier each for P^T and dS^T (the warpgroups
-can finish tile i + 1 before the MMA thread has waited for tile i), an S MMA
-issued without waiting for the warpgroups to have read the previous S, and a
-P^T readiness arrival sent before P^T is written.
+The kernels' protocols pass at several ring depths, tile counts, item mixes
+and warpgroup counts.  Planted mistakes must be caught: the two-buffer dK/dV
+form with one readiness barrier each for P^T and dS^T (the warpgroups can
+finish tile i + 1 before the MMA thread has waited for tile i), an S MMA
+issued without waiting for the warpgroups to have read the previous S, a P^T
+readiness arrival sent before P^T is written, a resident slot of the
+persistent backward reloaded too early, and the persistent forward's first
+build, with one scores-ready barrier per TMEM buffer shared by both query
+tiles.
 """
 import random
 import re
@@ -77,7 +81,7 @@ class Model:
 
     def run(self, max_steps=500000):
         gens = dict(self.roles)
-        cur = {name: next(g) for name, g in gens.items()}
+        cur = {name: next(g, None) for name, g in gens.items()}
         for _ in range(max_steps):
             ready = []
             for name, op in cur.items():
@@ -587,3 +591,173 @@ def test_dkdv_persistent_protocol(items, SX, SY, NG):
 def test_resident_slot_reused_too_early_is_caught(roles):
     errs = _errors(lambda: roles([1, 1, 1, 2], 4, 4, 4, mistake="no_res_empty_wait"), 800)
     assert any(re.search(r"reads Res\d expecting R\d, finds R\d", e) for e in errs)
+
+
+# ---------------------------------------------------------------- persistent forward
+#
+# fwd_persist_sm100.cuh: items of one or two 128-row query tiles; units
+# u = (item, key tile j, query tile t), t fastest.  Unit u's scores go to TMEM
+# buffer u % NB; each warpgroup (t, c) evaluates half c of its tile's scores
+# and writes P over them; O_t += P V_j reads P from the buffer, and the MMA
+# thread issues the scores of unit u + NB right after it (same buffer).  Each
+# buffer has one scores-ready barrier per query tile; p_full[buffer] collects
+# the two warpgroups of the unit's tile; o_full[t] completes once per item that
+# has tile t, after which tile t's warpgroups read O_t.
+
+def fwd_persistent_roles(items, NB=3, NQ=2, KS=4, VS=4, mistake=None):
+    """items: (ntiles, nkv) per item of one block."""
+    units = [(n, j, t) for n, (nt, nkv) in enumerate(items) for j in range(nkv) for t in range(nt)]
+    U = len(units)
+    one_sfull = mistake == "one_scores_barrier_per_buffer"
+
+    def s_bar(u):
+        n, j, t = units[u]
+        return f"s_full{u % NB}" if one_sfull else f"s_full{u % NB}.{t}"
+
+    def loadQK():
+        jk = 0
+        for n, (nt, nkv) in enumerate(items):
+            qs = n % NQ
+            if n >= NQ:
+                yield ("wait", f"q_empty{qs}", n // NQ - 1)
+            # the item's one or two query tiles land on one barrier: one load here
+            yield ("tma", f"q_full{qs}", n // NQ, f"Q{qs}", f"Q{n}")
+            for j in range(nkv):
+                ks = jk % KS
+                if jk >= KS:
+                    yield ("wait", f"k_empty{ks}", jk // KS - 1)
+                yield ("tma", f"k_full{ks}", jk // KS, f"K{ks}", f"K{n}.{j}")
+                jk += 1
+        for i in range(max(len(items) - NQ, 0), len(items)):
+            yield ("wait", f"q_full{i % NQ}", i // NQ)
+        for i in range(max(jk - KS, 0), jk):
+            yield ("wait", f"k_full{i % KS}", i // KS)
+
+    def loadV():
+        jv = 0
+        for n, (nt, nkv) in enumerate(items):
+            for j in range(nkv):
+                vs = jv % VS
+                if jv >= VS:
+                    yield ("wait", f"v_empty{vs}", jv // VS - 1)
+                yield ("tma", f"v_full{vs}", jv // VS, f"V{vs}", f"V{n}.{j}")
+                jv += 1
+        for i in range(max(jv - VS, 0), jv):
+            yield ("wait", f"v_full{i % VS}", i // VS)
+
+    # ring indices of each unit: item n's query slot, key / value index of (n, j)
+    kv_index = {}
+    for n, (nt, nkv) in enumerate(items):
+        for j in range(nkv):
+            kv_index[(n, j)] = len(kv_index)
+    uses = {}   # scores-barrier completions so far, per barrier
+
+    def issue_s(u):
+        n, j, t = units[u]
+        nt, nkv = items[n]
+        q = kv_index[(n, j)]
+        if j == 0 and t == 0:
+            yield ("wait", f"q_full{n % NQ}", n // NQ)
+        if t == 0:
+            yield ("wait", f"k_full{q % KS}", q // KS)
+        b = u % NB
+        yield ("mma", [(f"Q{n % NQ}", f"Q{n}"), (f"K{q % KS}", f"K{n}.{j}")],
+               [(f"S{b}.0", f"S{u}"), (f"S{b}.1", f"S{u}")])
+        bar = s_bar(u)
+        yield ("commit", bar, uses.get(bar, 0))
+        uses[bar] = uses.get(bar, 0) + 1
+        if t == nt - 1:
+            yield ("commit", f"k_empty{q % KS}", q // KS)
+            if j == nkv - 1:
+                yield ("commit", f"q_empty{n % NQ}", n // NQ)
+
+    def mma():
+        for u in range(min(NB, U)):
+            yield from issue_s(u)
+        seen_o = [0, 0]
+        for u in range(U):
+            n, j, t = units[u]
+            nt, nkv = items[n]
+            q = kv_index[(n, j)]
+            if t == 0:
+                yield ("wait", f"v_full{q % VS}", q // VS)
+            yield ("wait", f"p_full{u % NB}", u // NB)
+            b = u % NB
+            yield ("mma", [(f"S{b}.0", f"P{u}"), (f"S{b}.1", f"P{u}"), (f"V{q % VS}", f"V{n}.{j}")] +
+                   ([(f"O{t}", f"O{n}.{j - 1}")] if j else []), [(f"O{t}", f"O{n}.{j}")])
+            if t == nt - 1:
+                yield ("commit", f"v_empty{q % VS}", q // VS)
+            if j == nkv - 1:
+                yield ("commit", f"o_full{t}", seen_o[t])
+                seen_o[t] += 1
+            if u + NB < U:
+                yield from issue_s(u + NB)
+        yield ("commit", "drain", 0)
+        yield ("wait", "drain", 0)
+
+    def sigma(t, c):
+        used = {}
+        no = 0
+        for u in range(U):
+            n, j, tt = units[u]
+            if tt != t:
+                continue
+            bar = s_bar(u)
+            if one_sfull:
+                # the first build: each tile counted its own uses of the buffer
+                key = f"{u % NB}"
+            else:
+                key = bar
+            ph = used.get(key, 0)
+            used[key] = ph + 1
+            yield ("wait", bar, ph)
+            b = u % NB
+            yield ("use", f"S{b}.{c}", f"S{u}")
+            yield ("write", f"S{b}.{c}", f"P{u}")
+            yield ("arrive", f"p_full{b}", u // NB)
+            nt, nkv = items[n]
+            if j == nkv - 1:
+                yield ("wait", f"o_full{t}", no)
+                no += 1
+                yield ("use", f"O{t}", f"O{n}.{j}")
+
+    bars = {"drain": 1, "o_full0": 1, "o_full1": 1}
+    for s in range(NQ):
+        bars[f"q_full{s}"] = 1
+        bars[f"q_empty{s}"] = 1
+    for s in range(KS):
+        bars[f"k_full{s}"] = 1
+        bars[f"k_empty{s}"] = 1
+    for s in range(VS):
+        bars[f"v_full{s}"] = 1
+        bars[f"v_empty{s}"] = 1
+    for b in range(NB):
+        bars[f"p_full{b}"] = 2          # the two warpgroups of the unit's tile
+        if one_sfull:
+            bars[f"s_full{b}"] = 1
+        else:
+            bars[f"s_full{b}.0"] = 1
+            bars[f"s_full{b}.1"] = 1
+    roles = {"loadQK": loadQK(), "loadV": loadV(), "mma": mma()}
+    roles.update({f"sigma{t}{c}": sigma(t, c) for t in range(2) for c in range(2)})
+    return bars, roles
+
+
+FWD_ITEMS = [[(2, 3)], [(1, 2)], [(2, 1), (1, 1), (2, 2)], [(1, 3), (2, 2), (1, 1), (1, 2)],
+             [(2, 4), (2, 1), (1, 3)], [(1, 1)] * 5]
+
+
+@pytest.mark.parametrize("items", FWD_ITEMS, ids=lambda it: "-".join(f"{a}x{b}" for a, b in it))
+@pytest.mark.parametrize("NB", [2, 3])
+def test_fwd_persistent_protocol(items, NB):
+    _explore(lambda: fwd_persistent_roles(items, NB=NB), 150)
+
+
+def test_fwd_one_scores_barrier_per_buffer_is_caught():
+    """The persistent forward's first build kept one scores-ready barrier per
+    TMEM buffer: with one- and two-tile items mixed, a tile that sits out some
+    units waits on a phase the other tile has already moved past."""
+    errs = _errors(lambda: fwd_persistent_roles([(2, 2), (1, 2), (2, 1), (1, 1)],
+                                                mistake="one_scores_barrier_per_buffer"), 800)
+    assert any(re.search(r"sigma\d\d waits for phase \d+ of s_full\d, which has completed|"
+                         r"reads S\d\.\d expecting S\d+, finds|deadlock", e) for e in errs)
