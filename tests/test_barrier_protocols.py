@@ -1,6 +1,6 @@
-"""Host-side model check of the kernels' barrier protocols: the backward
-tile kernels (bwd_sm100.cuh), the persistent backward (bwd_persist_sm100.cuh)
-and the persistent forward (fwd_persist_sm100.cuh).
+"""Host-side model check of the kernels' barrier protocols: the forward and
+backward tile kernels (fwd_sm100.cuh, bwd_sm100.cuh), the persistent backward
+(bwd_persist_sm100.cuh) and the persistent forward (fwd_persist_sm100.cuh).
 
 Each role of a block (the TMA producers, the MMA issuer, the sigma
 warpgroups) is written as the sequence of barrier waits, arrivals, tensor-core
@@ -761,3 +761,92 @@ def test_fwd_one_scores_barrier_per_buffer_is_caught():
                                                 mistake="one_scores_barrier_per_buffer"), 800)
     assert any(re.search(r"sigma\d\d waits for phase \d+ of s_full\d, which has completed|"
                          r"reads S\d\.\d expecting S\d+, finds|deadlock", e) for e in errs)
+
+
+# ---------------------------------------------------------------- tile forward (D = 128)
+#
+# fwd_sm100.cuh: one block per pair of query tiles.  S_t (scores of tile t)
+# lives in its own TMEM buffer; per key tile j the MMA thread issues
+# O_t += P_t V_j as tile t's warpgroups publish P_t (p_full[t]) and then S_t
+# of key tile j + 1 into the same buffer (MMAs run in issue order).
+
+def fwd_tiles_roles(ntiles, nkv, KS=2, VS=3, mistake=None):
+    def loadQK():
+        yield ("tma", "q_full", 0, "Q", "Q")
+        for j in range(nkv):
+            if j >= KS:
+                yield ("wait", f"k_empty{j % KS}", j // KS - 1)
+            yield ("tma", f"k_full{j % KS}", j // KS, f"K{j % KS}", f"K{j}")
+        yield ("wait", "q_full", 0)
+        for j in range(max(nkv - KS, 0), nkv):
+            yield ("wait", f"k_full{j % KS}", j // KS)
+
+    def loadV():
+        for j in range(nkv):
+            if j >= VS:
+                yield ("wait", f"v_empty{j % VS}", j // VS - 1)
+            yield ("tma", f"v_full{j % VS}", j // VS, f"V{j % VS}", f"V{j}")
+        for j in range(max(nkv - VS, 0), nkv):
+            yield ("wait", f"v_full{j % VS}", j // VS)
+
+    def issue_s(t, j):
+        yield ("mma", [("Q", "Q"), (f"K{j % KS}", f"K{j}")], [(f"S{t}.0", f"S{t}:{j}"), (f"S{t}.1", f"S{t}:{j}")])
+        yield ("commit", f"s_full{t}", j)
+
+    def mma():
+        yield ("wait", "q_full", 0)
+        yield ("wait", "k_full0", 0)
+        for t in range(ntiles):
+            yield from issue_s(t, 0)
+        yield ("commit", "k_empty0", 0)
+        for j in range(nkv):
+            more = j + 1 < nkv
+            yield ("wait", f"v_full{j % VS}", j // VS)
+            for t in range(ntiles):
+                if mistake != "no_p_wait":
+                    yield ("wait", f"p_full{t}", j)
+                yield ("mma", [(f"S{t}.0", f"P{t}:{j}"), (f"S{t}.1", f"P{t}:{j}"), (f"V{j % VS}", f"V{j}")] +
+                       ([(f"O{t}", f"O{t}:{j - 1}")] if j else []), [(f"O{t}", f"O{t}:{j}")])
+                if t == ntiles - 1:
+                    yield ("commit", f"v_empty{j % VS}", j // VS)
+                if more:
+                    if t == 0:
+                        yield ("wait", f"k_full{(j + 1) % KS}", (j + 1) // KS)
+                    yield from issue_s(t, j + 1)
+                    if t == ntiles - 1:
+                        yield ("commit", f"k_empty{(j + 1) % KS}", (j + 1) // KS)
+        yield ("commit", "drain", 0)
+        yield ("wait", "drain", 0)
+
+    def sigma(t, c):
+        if t >= ntiles:
+            return
+        for j in range(nkv):
+            yield ("wait", f"s_full{t}", j)
+            yield ("use", f"S{t}.{c}", f"S{t}:{j}")
+            yield ("write", f"S{t}.{c}", f"P{t}:{j}")
+            yield ("arrive", f"p_full{t}", j)
+        yield ("wait", "drain", 0)
+        yield ("use", f"O{t}", f"O{t}:{nkv - 1}")
+
+    bars = {"q_full": 1, "drain": 1, "s_full0": 1, "s_full1": 1, "p_full0": 2, "p_full1": 2}
+    for s in range(KS):
+        bars[f"k_full{s}"] = 1
+        bars[f"k_empty{s}"] = 1
+    for s in range(VS):
+        bars[f"v_full{s}"] = 1
+        bars[f"v_empty{s}"] = 1
+    roles = {"loadQK": loadQK(), "loadV": loadV(), "mma": mma()}
+    roles.update({f"sigma{t}{c}": sigma(t, c) for t in range(2) for c in range(2)})
+    return bars, roles
+
+
+@pytest.mark.parametrize("ntiles", [1, 2])
+@pytest.mark.parametrize("nkv", [1, 2, 3, 6])
+def test_fwd_tiles_protocol(ntiles, nkv):
+    _explore(lambda: fwd_tiles_roles(ntiles, nkv), 150)
+
+
+def test_fwd_tiles_missing_p_wait_is_caught():
+    errs = _errors(lambda: fwd_tiles_roles(2, 3, mistake="no_p_wait"), 800)
+    assert any(re.search(r"an MMA reads S\d\.\d expecting P\d:\d, finds S\d:\d", e) for e in errs)
