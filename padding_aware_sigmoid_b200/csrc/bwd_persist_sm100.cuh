@@ -225,8 +225,9 @@ struct BwdUnits {
 };
 
 // Streams one ring (S slots) over every item of the walk, after the resident
-// tiles of each item when `res` is set.  Returns the loads issued; `res_n`
-// receives the resident loads issued.
+// tiles of each item when `res` is set.  `issued` receives the ring loads
+// issued and `res_n` the resident loads issued (both stop early when a wait
+// gives up), for the drain before the CTA exits.
 template <int S, int NSUB>
 __device__ __forceinline__ void bwd_persistent_producer(const CUtensorMap *map, uint64_t *full, uint64_t *empty,
                                                         uint8_t *ring, int tile_bytes, BwdWalk walk,
