@@ -252,8 +252,10 @@ sigattn_status sigattn_sigmoid_eval(const float *x, float *y, float *dy, int64_t
 sigattn_status sigattn_last_device_status(void *stream);
 
 /* Bound, in nanoseconds, on every wait inside the bf16 kernels (default
- * 4e9).  A wait that runs out records SIGATTN_ERR_TIMEOUT, the kernel
- * abandons its work, frees its tensor memory and exits. */
+ * 4e9, at least 1e6, else SIGATTN_ERR_INVALID_ARG).  A wait that runs out
+ * records SIGATTN_ERR_TIMEOUT, the kernel abandons its work, waits (with the
+ * same bound) for the tile loads and MMAs it has in flight, frees its tensor
+ * memory and exits. */
 sigattn_status sigattn_set_wait_timeout_ns(uint64_t ns);
 
 /* Launches a one-CTA kernel whose only job is to wait on a barrier that

@@ -30,6 +30,7 @@ int g_cc_major[kMaxDevices] = {};         // 0 = not queried yet
 int g_sm_count[kMaxDevices] = {};         // multiprocessors per device (persistent grids)
 std::atomic<int> g_sigmoid_mode{kSigmoidTanh};
 std::atomic<uint64_t> g_timeout_ns{4000000000ull};
+constexpr uint64_t kMinWaitTimeoutNs = 1000000ull;   // 1 ms
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_last_cuda_error{0};
 
@@ -737,7 +738,10 @@ sigattn_status sigattn_last_device_status(void *stream) {
 }
 
 sigattn_status sigattn_set_wait_timeout_ns(uint64_t ns) {
-    if (ns == 0) return SIGATTN_ERR_INVALID_ARG;
+    // the same bound limits the waits with which a block, after a wait ran
+    // out, lets its in-flight tile loads and MMAs land before it releases its
+    // shared and tensor memory: those take microseconds, so 1 ms is the floor
+    if (ns < kMinWaitTimeoutNs) return SIGATTN_ERR_INVALID_ARG;
     g_timeout_ns.store(ns);
     return SIGATTN_OK;
 }

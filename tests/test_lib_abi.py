@@ -79,6 +79,8 @@ def test_host_validation_needs_no_gpu(lib):
     assert lib.sigattn_set_sigmoid_mode(0) == 0 and lib.sigattn_get_sigmoid_mode() == 0
     assert lib.sigattn_set_sigmoid_mode(old) == 0
     assert lib.sigattn_set_wait_timeout_ns(0) == 1
+    # below 1 ms the bound would also cut short the waits for in-flight loads
+    assert lib.sigattn_set_wait_timeout_ns(999_999) == 1
 
 
 def test_bias_entry_points_host_validation(lib):
