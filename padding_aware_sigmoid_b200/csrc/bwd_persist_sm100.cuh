@@ -225,7 +225,9 @@ struct BwdUnits {
 };
 
 // Streams one ring (S slots) over every item of the walk, after the resident
-// tiles of each item when `res` is set.  `issued` receives the ring loads
+// tiles of each item when `res` is set.  The whole warp runs it converged: all
+// lanes wait, lane 0 arms the barrier and issues the copies (0.5-1% faster
+// than one lane of a diverged warp).  `issued` receives the ring loads
 // issued and `res_n` the resident loads issued (both stop early when a wait
 // gives up), for the drain before the CTA exits.
 template <int S, int NSUB>
@@ -235,28 +237,36 @@ __device__ __forceinline__ void bwd_persistent_producer(const CUtensorMap *map, 
                                                         uint64_t *res_full, uint64_t *res_empty, uint8_t *res,
                                                         const WaitCtx &wctx, int &issued, int &res_n) {
     constexpr int SUB = 128 * 64 * 2;
+    const bool leader = lane_id() == 0;
     BwdItem it;
     int q = 0, k = 0;
     bool ok = true;
     while (ok && walk.next(it)) {
         if (res != nullptr) {
             const int rs = k & 1;
-            if (k >= 2 && !(ok = mbar_wait(&res_empty[rs], ((k >> 1) - 1) & 1, wctx))) break;
-            mbar_arrive_expect_tx(&res_full[rs], 2 * tile_bytes);
-            for (int s = 0; s < NSUB; ++s) {
-                tma_load_4d(res_a, &res_full[rs], res + (2 * rs) * tile_bytes + s * SUB, 64 * s, it.h,
-                            it.tile * 128, it.z);
-                tma_load_4d(res_b, &res_full[rs], res + (2 * rs + 1) * tile_bytes + s * SUB, 64 * s, it.h,
-                            it.tile * 128, it.z);
+            if (k >= 2 && !(ok = __all_sync(0xffffffffu, mbar_wait(&res_empty[rs], ((k >> 1) - 1) & 1, wctx))))
+                break;
+            if (leader) {
+                mbar_arrive_expect_tx(&res_full[rs], 2 * tile_bytes);
+                for (int s = 0; s < NSUB; ++s) {
+                    tma_load_4d(res_a, &res_full[rs], res + (2 * rs) * tile_bytes + s * SUB, 64 * s, it.h,
+                                it.tile * 128, it.z);
+                    tma_load_4d(res_b, &res_full[rs], res + (2 * rs + 1) * tile_bytes + s * SUB, 64 * s, it.h,
+                                it.tile * 128, it.z);
+                }
             }
+            __syncwarp();
             ++k;
         }
         for (int j = 0; j < it.nsteps; ++j) {
             const int st = q % S;
-            if (q >= S && !(ok = mbar_wait(&empty[st], ((q / S) - 1) & 1, wctx))) break;
-            mbar_arrive_expect_tx(&full[st], tile_bytes);
-            for (int s = 0; s < NSUB; ++s)
-                tma_load_4d(map, &full[st], ring + st * tile_bytes + s * SUB, 64 * s, it.h, j * 128, it.z);
+            if (q >= S && !(ok = __all_sync(0xffffffffu, mbar_wait(&empty[st], ((q / S) - 1) & 1, wctx)))) break;
+            if (leader) {
+                mbar_arrive_expect_tx(&full[st], tile_bytes);
+                for (int s = 0; s < NSUB; ++s)
+                    tma_load_4d(map, &full[st], ring + st * tile_bytes + s * SUB, 64 * s, it.h, j * 128, it.z);
+            }
+            __syncwarp();
             ++q;
         }
     }
@@ -384,7 +394,7 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
     const BwdWalk walk0{&p, table, meta[0], p.Z <= kBwdMaxRanked, true, 0};
 
     if (warp == 0) {
-        if (lane == 0) {
+        {
             int issued, res_n;
             bwd_persistent_producer<SX, Lay::NSUB>(&tmK, x_full, x_empty, smem + Lay::OFF_X, Lay::TILE_BYTES,
                                                    walk0, &tmQ, &tmDO, res_full, res_empty, smem + Lay::OFF_R,
@@ -393,7 +403,7 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
         }
     } else if (warp == 2) {
         // V_j ring, fed by its own thread so it never waits behind a key slot
-        if (lane == 0) {
+        {
             int issued, res_n;
             bwd_persistent_producer<SY, Lay::NSUB>(&tmV, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
                                                    walk0, nullptr, nullptr, nullptr, nullptr, nullptr, wctx,
@@ -620,7 +630,7 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
     const BwdWalk walk0{&p, table, meta[0], p.Z <= kBwdMaxRanked, false, 0};
 
     if (warp == 0) {
-        if (lane == 0) {
+        {
             int issued, res_n;
             bwd_persistent_producer<SX, Lay::NSUB>(&tmQ, x_full, x_empty, smem + Lay::OFF_X, Lay::TILE_BYTES,
                                                    walk0, &tmK, &tmV, res_full, res_empty, smem + Lay::OFF_R,
@@ -628,7 +638,7 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
             bwd_persistent_drain<SX>(x_full, issued, res_full, res_n, p.timeout_ns);
         }
     } else if (warp == 2) {
-        if (lane == 0) {
+        {
             int issued, res_n;
             bwd_persistent_producer<SY, Lay::NSUB>(&tmDO, y_full, y_empty, smem + Lay::OFF_Y, Lay::TILE_BYTES,
                                                    walk0, nullptr, nullptr, nullptr, nullptr, nullptr, wctx,
