@@ -13,7 +13,8 @@
 // Warp roles (640 threads):
 //   warp 0       TMA producer: Q tiles once, then K_j into the key ring
 //   warp 2       TMA producer: V_j into the value ring
-//   warp 1       owns TMEM; one thread issues every tcgen05.mma
+//   warp 1       owns TMEM and issues every tcgen05.mma, the whole warp running
+//                converged (elect.sync picks the issuing lane)
 //   warp 3       idle
 //   warps 4-19   four sigma warpgroups (thread = query row = TMEM lane):
 //                warpgroup g serves query tile t = g / 2, key columns
@@ -217,7 +218,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        {
+            // the whole warp runs converged; elect.sync picks the issuing lane
+            auto wt = [&](uint64_t *bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, wctx));
+            };
             const uint32_t idesc_s = idesc_bf16_f32(128, Lay::BN, false, false);
             const uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
             const uint32_t sQ = smem_u32(smem + Lay::OFF_Q);
@@ -230,10 +235,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                    mma_ss(d_tmem, smem_desc_sw128(qbase + koff, 16, 1024),
+                    mma_ss_w(d_tmem, smem_desc_sw128(qbase + koff, 16, 1024),
                            smem_desc_sw128(kbase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&s_full[t]);
+                mma_commit_w(&s_full[t]);
             };
             // O_t += P_t V_j, P_t read from TMEM (16 keys = 8 packed columns per step;
             // keys 64-127 sit 32 columns further on, see the sigma warpgroups)
@@ -242,7 +247,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const uint32_t a_tmem = tmem + (t ? Lay::COL_S1 : Lay::COL_S0);
 #pragma unroll
                 for (int kk = 0; kk < Lay::BN / 16; ++kk)
-                    mma_ts(d_tmem, a_tmem + kk * 8 + (kk >= 4 ? 32 : 0),
+                    mma_ts_w(d_tmem, a_tmem + kk * 8 + (kk >= 4 ? 32 : 0),
                            smem_desc_sw128(vbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_o,
                            (!first || kk > 0) ? 1u : 0u);
             };
@@ -252,11 +257,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // j+1 overwrites P_t of j right after O_t += P_t V_j is issued: MMAs
             // issued by one thread execute in issue order, so the P.V MMA has read
             // P_t before the next scores are written over it.
-            bool ok = mbar_wait(q_full, 0, wctx) && mbar_wait(&k_full[0], 0, wctx);
+            bool ok = wt(q_full, 0) && wt(&k_full[0], 0);
             if (ok) {
                 tc_fence_after();
                 for (int t = 0; t < ntiles; ++t) issue_s(t, sK);
-                mma_commit(&k_empty[0]);
+                mma_commit_w(&k_empty[0]);
             }
             for (int j = 0; ok && j < nkv; ++j) {
                 const int stv = j % VS;
@@ -264,27 +269,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const bool more = j + 1 < nkv;
                 const uint32_t vbase = sV + stv * Lay::TILE_BYTES;
                 const uint32_t knext = sK + stk * Lay::TILE_BYTES;
-                if (!(ok = mbar_wait(&v_full[stv], (j / VS) & 1, wctx))) break;
+                if (!(ok = wt(&v_full[stv], (j / VS) & 1))) break;
                 trace(1, j, 0);
                 for (int t = 0; t < ntiles; ++t) {
-                    if (!(ok = mbar_wait(&p_full[t], j & 1, wctx))) break;
+                    if (!(ok = wt(&p_full[t], j & 1))) break;
                     trace(1, j, 1 + 3 * t);
                     tc_fence_after();
                     issue_pv(t, vbase, j == 0);
                     trace(1, j, 2 + 3 * t);
-                    if (t == ntiles - 1) mma_commit(&v_empty[stv]);
+                    if (t == ntiles - 1) mma_commit_w(&v_empty[stv]);
                     if (more) {
-                        if (t == 0 && !(ok = mbar_wait(&k_full[stk], ((j + 1) / KS) & 1, wctx))) break;
+                        if (t == 0 && !(ok = wt(&k_full[stk], ((j + 1) / KS) & 1))) break;
                         tc_fence_after();
                         issue_s(t, knext);
                         trace(1, j, 3 + 3 * t);
-                        if (t == ntiles - 1) mma_commit(&k_empty[stk]);
+                        if (t == ntiles - 1) mma_commit_w(&k_empty[stk]);
                     }
                 }
             }
             // No MMA may still be running when TMEM is released.
-            mma_commit(drain);
+            mma_commit_w(drain);
             mbar_wait_drain(drain, 0, p.timeout_ns);
+            __syncwarp();
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ sigma warpgroups
