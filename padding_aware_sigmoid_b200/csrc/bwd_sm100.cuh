@@ -749,21 +749,23 @@ __global__ void __launch_bounds__(BwdSigma<D>::kThreads, 1)
             const uint32_t xring = smem_u32(smem + Lay::OFF_X), yring = smem_u32(smem + Lay::OFF_Y);
             auto qslot = [&](int i) { return xring + (i % SX) * Lay::TILE_BYTES; };
             auto doslot = [&](int i) { return yring + (i % SY) * Lay::TILE_BYTES; };
+            // descriptors as low words (start and LBO) plus the K step's offset >> 4
+            constexpr uint32_t kDescHi = desc_hi(1024);
             auto issue_xyT = [&](uint32_t col, uint32_t xbase, uint32_t ybase) {
+                const uint32_t x_lo = desc_lo(xbase, 16), y_lo = desc_lo(ybase, 16);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32;
-                    mma_ss_w(tmem + col, smem_desc_sw128(xbase + koff, 16, 1024),
-                             smem_desc_sw128(ybase + koff, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t koff = ((kk >> 2) * Lay::SUB_BYTES + (kk & 3) * 32) >> 4;
+                    mma_ss_lhw(tmem + col, x_lo + koff, y_lo + koff, kDescHi, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // acc += A(TMEM, packed over `acol`) * B (128 query rows, MN-major)
             auto issue_acc = [&](uint32_t acc, uint32_t acol, uint32_t bbase, bool first) {
+                const uint32_t b_lo = desc_lo(bbase, Lay::SUB_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts_w(tmem + acc, tmem + acol + BwdSigma<D>::packed_col(kk),
-                             smem_desc_sw128(bbase + kk * 16 * 128, Lay::SUB_BYTES, 1024), idesc_kv,
-                             (!first || kk > 0) ? 1u : 0u);
+                    mma_ts_lhw(tmem + acc, tmem + acol + BwdSigma<D>::packed_col(kk), b_lo + kk * ((16 * 128) >> 4),
+                               kDescHi, idesc_kv, (!first || kk > 0) ? 1u : 0u);
             };
             bool ok = wait(res_full, 0) && wait(&x_full[0], 0) && wait(&y_full[0], 0);
             if (ok) {
